@@ -1,0 +1,141 @@
+/*
+ * sta.h - C ABI of the B200 (sm_100a) Sliding Tile Attention forward library.
+ *
+ * Method: "Fast Video Generation with Sliding Tile Attention" (arXiv 2502.04507).
+ *   - abstract: attention restricted to a local 3D window that moves tile by
+ *     tile rather than token by token;
+ *   - summary page, "Method details": the latent video (T, H, W) is cut into
+ *     non-overlapping (tt, th, tw) tiles whose tokens are made contiguous, so
+ *     attention between a query tile and a key tile is a dense block;
+ *   - summary page, "Core innovation": blocks are fully attended or skipped;
+ *     "Technical contribution": the window is set per attention head;
+ *   - review reply on input resolution: tile (6, 8, 8); latent dimensions must
+ *     be multiples of the tile.
+ * Window rule: query tile a attends key tile k iff, in every dimension x,
+ *   s_x <= k_x < s_x + w'_x  with  w'_x = min(w_x, n_x)  and
+ *   s_x = clamp(a_x - floor(w'_x / 2), 0, n_x - w'_x),
+ * n_x being the number of tiles in dimension x and w_x the head's window, in
+ * tiles.  A window wider than the grid therefore covers the grid.
+ *
+ * Layout conventions (all entry points):
+ *   - every q/k/v/out tensor is a contiguous bf16 array [batch, heads, L, d]
+ *     (row-major, d fastest), L = T * H * W tokens, d in {64, 128};
+ *   - raster order: token n = (t * H + h) * W + w;
+ *   - tiled order: tiles in raster order over the tile grid, tokens in raster
+ *     order inside a tile; tile i occupies rows [i * Ntile, (i + 1) * Ntile).
+ *
+ * Ownership and execution: the caller owns every device buffer.  Calls are
+ * asynchronous on the given stream (a cudaStream_t passed as void*, NULL = the
+ * legacy default stream), out of place, and never synchronise unless stated.
+ * On an invalid argument a call returns an error before touching any buffer or
+ * the device.  Nothing is printed.
+ */
+#ifndef STA_H_
+#define STA_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct {
+  int32_t t, h, w;
+} sta_dim3;
+
+typedef enum {
+  STA_OK = 0,
+  STA_ERR_NULL = 1,      /* a required pointer is NULL */
+  STA_ERR_ALIGN = 2,     /* a device pointer is not 16-byte aligned */
+  STA_ERR_ALIAS = 3,     /* an output overlaps an input */
+  STA_ERR_SHAPE = 4,     /* grid/tile not positive, grid not a multiple of the tile, sizes too large */
+  STA_ERR_WINDOW = 5,    /* a window dimension is < 1 */
+  STA_ERR_HEADDIM = 6,   /* d is not 64 or 128 */
+  STA_ERR_ARCH = 7,      /* the current device is not compute capability 10.0 (B200) */
+  STA_ERR_CUDA = 8,      /* a CUDA runtime/driver call failed (message via sta_last_cuda_error) */
+  STA_ERR_TIMEOUT = 9,   /* a kernel's bounded wait expired; the kernel gave up */
+  STA_ERR_ARG = 10       /* another argument is out of range (batch, heads, scale not finite ...) */
+} sta_status;
+
+/* Human-readable name of a status code.  Static storage; never NULL. */
+const char* sta_status_str(sta_status s);
+
+/* Text of the last CUDA error seen by this thread inside the library ("" if none). */
+const char* sta_last_cuda_error(void);
+
+/*
+ * Index map raster -> tiled (host only, no device use).
+ *   tiled_of_raster: host array of L = T*H*W int32 written by the call;
+ *   tiled_of_raster[n] is the tiled row of raster token n.
+ * Errors: STA_ERR_NULL, STA_ERR_SHAPE.
+ */
+sta_status sta_tile_index_map(sta_dim3 grid, sta_dim3 tile, int32_t* tiled_of_raster);
+
+/*
+ * Attended (query, key) token pairs summed over batch and heads (host only):
+ *   batch * sum_h L * Ntile * prod_x min(w_h,x, n_x).
+ * FLOPs of the forward pass are 4 * d * pairs.  windows: host array of `heads`
+ * entries.  Returns -1 on an invalid argument.
+ */
+int64_t sta_attended_pairs(int32_t batch, int32_t heads, sta_dim3 grid, sta_dim3 tile,
+                           const sta_dim3* windows);
+
+/*
+ * Reorder raster -> tiled (summary page, "Method details": tokens of a tile made
+ * contiguous).  src, dst: device bf16 [batch_heads, L, d], 16-byte aligned, not
+ * overlapping.  dst[bh, tiled(n), :] = src[bh, n, :], bit-exact.
+ * HBM-bound gather of d*2-byte rows with 16-byte vector accesses.
+ * Errors: NULL, ALIGN, ALIAS, SHAPE, HEADDIM, ARG, ARCH, CUDA.
+ */
+sta_status sta_tile_reorder(const void* src, void* dst, int64_t batch_heads, int32_t d,
+                            sta_dim3 grid, sta_dim3 tile, void* stream);
+
+/* Inverse of sta_tile_reorder: dst[bh, n, :] = src[bh, tiled(n), :]. */
+sta_status sta_tile_unorder(const void* src, void* dst, int64_t batch_heads, int32_t d,
+                            sta_dim3 grid, sta_dim3 tile, void* stream);
+
+/*
+ * STA forward on tiled-order tensors (abstract; "Method details"; "Core
+ * innovation"): for every head h and query token i,
+ *   out[i] = sum_j softmax_j(scale * q_i . k_j) v_j
+ * over the key tokens j whose tile lies in the window of i's tile (rule above,
+ * window_per_head[h]).  q, k, v, out: device bf16 [batch, heads, L, d] in tiled
+ * order, 16-byte aligned; out must not overlap q, k or v.  window_per_head:
+ * host array of `heads` windows in tiles, read during the call only.
+ * Arithmetic: bf16 inputs, fp32 tensor-core accumulation, fp32 online softmax,
+ * probabilities rounded to bf16 for the P*V product, output rounded to bf16.
+ * The first call with a new (batch, heads, grid, tile, windows) builds and
+ * uploads a work schedule synchronously (do it before any stream capture);
+ * later calls reuse it.  Kernel timeouts are reported by
+ * sta_check_device_status.
+ * Errors: NULL, ALIGN, ALIAS, SHAPE, WINDOW, HEADDIM, ARG, ARCH, CUDA.
+ */
+sta_status sta_attention_fwd(const void* q, const void* k, const void* v, void* out,
+                             int32_t batch, int32_t heads, int32_t d, sta_dim3 grid,
+                             sta_dim3 tile, const sta_dim3* window_per_head, float scale,
+                             void* stream);
+
+/*
+ * Synchronises `stream` and reports whether any kernel of this library gave up
+ * on a bounded wait since the last check (STA_ERR_TIMEOUT), then clears the
+ * flag.  Returns STA_ERR_CUDA if the stream has a pending CUDA error.
+ */
+sta_status sta_check_device_status(void* stream);
+
+/*
+ * Self-test of the bounded-wait path: launches one block whose threads wait on
+ * a shared-memory barrier that nothing completes, with a limit of `limit_ns`
+ * nanoseconds (clamped to [1e5, 5e9]), and synchronises `stream`.  A correct
+ * library returns STA_ERR_TIMEOUT and leaves the context usable.  No schedule
+ * or tensor is touched.
+ */
+sta_status sta_selftest_bounded_wait(uint64_t limit_ns, void* stream);
+
+/* Releases the library's cached schedules and device workspaces (all devices). */
+void sta_shutdown(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* STA_H_ */

@@ -88,8 +88,10 @@ def sta_mask(q_coords: np.ndarray, k_coords: np.ndarray, grid, tile, window) -> 
     qa = np.asarray(q_coords) // tsz
     ka = np.asarray(k_coords) // tsz
     start = window_start(qa, weff, ntiles)
-    inside = (ka[None, :, :] >= start[:, None, :]) & (ka[None, :, :] < (start + weff)[:, None, :])
-    return inside.all(axis=-1)
+    mask = np.ones((qa.shape[0], ka.shape[0]), dtype=bool)
+    for x in range(3):  # inside the window in every dimension
+        mask &= (ka[None, :, x] >= start[:, None, x]) & (ka[None, :, x] < start[:, None, x] + weff[x])
+    return mask
 
 
 def masked_softmax_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, mask: np.ndarray,
@@ -109,7 +111,7 @@ def masked_softmax_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, mask: 
 
 def sta_attention_head(q: np.ndarray, k: np.ndarray, v: np.ndarray, grid, tile, window,
                        scale: float, rows: Optional[Iterable[int]] = None,
-                       row_block: int = 512) -> np.ndarray:
+                       row_block: Optional[int] = None) -> np.ndarray:
     """STA forward of one (batch, head): q, k, v are [L, d] in raster order.
 
     Returns fp64 output rows for ``rows`` (all rows when None), in that order.
@@ -121,6 +123,8 @@ def sta_attention_head(q: np.ndarray, k: np.ndarray, v: np.ndarray, grid, tile, 
     if coords.shape[0] != L:
         raise ValueError("q rows do not match the grid")
     rows = np.arange(L) if rows is None else np.asarray(list(rows), dtype=np.int64)
+    if row_block is None:
+        row_block = int(min(512, max(16, (1 << 19) // L)))
     out = np.empty((rows.shape[0], v.shape[1]), dtype=np.float64)
     k64 = np.asarray(k, dtype=np.float64)
     v64 = np.asarray(v, dtype=np.float64)

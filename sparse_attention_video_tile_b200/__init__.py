@@ -1,0 +1,217 @@
+"""Python binding of the B200 Sliding Tile Attention library (``libsta.so``).
+
+Argument marshalling only: every step of the computation runs in the library's
+CUDA kernels.  The functions carry the names of the C entry points declared in
+``include/sta.h`` and take torch tensors (device memory owned by the caller) and
+the current torch CUDA stream.  There is no fallback: if the library is missing
+or the device is not a B200, the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence, Tuple
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsta.so")
+
+STATUS_NAMES = {
+    0: "STA_OK", 1: "STA_ERR_NULL", 2: "STA_ERR_ALIGN", 3: "STA_ERR_ALIAS", 4: "STA_ERR_SHAPE",
+    5: "STA_ERR_WINDOW", 6: "STA_ERR_HEADDIM", 7: "STA_ERR_ARCH", 8: "STA_ERR_CUDA",
+    9: "STA_ERR_TIMEOUT", 10: "STA_ERR_ARG",
+}
+STA_OK, STA_ERR_TIMEOUT = 0, 9
+
+
+class sta_dim3(ctypes.Structure):
+    _fields_ = [("t", ctypes.c_int32), ("h", ctypes.c_int32), ("w", ctypes.c_int32)]
+
+
+class StaError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str = ""):
+        self.status = status
+        msg = f"{where}: {STATUS_NAMES.get(status, status)}"
+        if detail:
+            msg += f" ({detail})"
+        super().__init__(msg)
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Loads libsta.so (built by ``sparse_attention_video_tile_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: run `python -m sparse_attention_video_tile_b200.build`")
+    lib = ctypes.CDLL(path)
+    P, I32, I64, U64, F = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint64, ctypes.c_float
+    D3 = sta_dim3
+    sigs = {
+        "sta_status_str": (ctypes.c_char_p, [ctypes.c_int]),
+        "sta_last_cuda_error": (ctypes.c_char_p, []),
+        "sta_tile_index_map": (ctypes.c_int, [D3, D3, ctypes.POINTER(ctypes.c_int32)]),
+        "sta_attended_pairs": (I64, [I32, I32, D3, D3, ctypes.POINTER(D3)]),
+        "sta_tile_reorder": (ctypes.c_int, [P, P, I64, I32, D3, D3, P]),
+        "sta_tile_unorder": (ctypes.c_int, [P, P, I64, I32, D3, D3, P]),
+        "sta_attention_fwd": (ctypes.c_int, [P, P, P, P, I32, I32, I32, D3, D3, ctypes.POINTER(D3), F, P]),
+        "sta_check_device_status": (ctypes.c_int, [P]),
+        "sta_selftest_bounded_wait": (ctypes.c_int, [U64, P]),
+        "sta_shutdown": (None, []),
+    }
+    for name, (res, args) in sigs.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def _d3(x: Sequence[int]) -> sta_dim3:
+    t = tuple(int(v) for v in x)
+    if len(t) != 3:
+        raise ValueError(f"expected (t, h, w), got {x!r}")
+    return sta_dim3(*t)
+
+
+def _windows(ws: Sequence[Sequence[int]]):
+    arr = (sta_dim3 * len(ws))()
+    for i, w in enumerate(ws):
+        arr[i] = _d3(w)
+    return arr
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(status: int, where: str) -> None:
+    if status != STA_OK:
+        detail = ""
+        if status == 8:
+            detail = load_library().sta_last_cuda_error().decode()
+        raise StaError(status, where, detail)
+
+
+def _tensor_ptr(x, name: str) -> int:
+    import torch
+    if not isinstance(x, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if x.dtype != torch.bfloat16:
+        raise TypeError(f"{name} must be bfloat16, got {x.dtype}")
+    if not x.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not x.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return x.data_ptr()
+
+
+def sta_status_str(status: int) -> str:
+    return load_library().sta_status_str(int(status)).decode()
+
+
+def sta_tile_index_map(grid, tile) -> np.ndarray:
+    """Raster -> tiled index map (int32 array of L entries)."""
+    L = int(np.prod([int(v) for v in grid]))
+    out = np.empty(L, dtype=np.int32)
+    st = load_library().sta_tile_index_map(_d3(grid), _d3(tile),
+                                           out.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)))
+    _check(st, "sta_tile_index_map")
+    return out
+
+
+def sta_attended_pairs(batch: int, heads: int, grid, tile, windows) -> int:
+    r = load_library().sta_attended_pairs(int(batch), int(heads), _d3(grid), _d3(tile), _windows(windows))
+    if r < 0:
+        raise StaError(10, "sta_attended_pairs")
+    return int(r)
+
+
+def sta_tile_reorder(src, dst, grid, tile, stream=None) -> None:
+    """dst[..., tiled(n), :] = src[..., n, :] for [.., L, d] bf16 CUDA tensors."""
+    d = int(src.shape[-1])
+    bh = int(src.numel() // (src.shape[-2] * d)) if src.numel() else 0
+    if tuple(dst.shape) != tuple(src.shape):
+        raise ValueError("src and dst shapes differ")
+    st = load_library().sta_tile_reorder(_tensor_ptr(src, "src"), _tensor_ptr(dst, "dst"), bh, d,
+                                         _d3(grid), _d3(tile), _stream(stream))
+    _check(st, "sta_tile_reorder")
+
+
+def sta_tile_unorder(src, dst, grid, tile, stream=None) -> None:
+    """dst[..., n, :] = src[..., tiled(n), :]."""
+    d = int(src.shape[-1])
+    bh = int(src.numel() // (src.shape[-2] * d)) if src.numel() else 0
+    if tuple(dst.shape) != tuple(src.shape):
+        raise ValueError("src and dst shapes differ")
+    st = load_library().sta_tile_unorder(_tensor_ptr(src, "src"), _tensor_ptr(dst, "dst"), bh, d,
+                                         _d3(grid), _d3(tile), _stream(stream))
+    _check(st, "sta_tile_unorder")
+
+
+def sta_attention_fwd(q, k, v, out, grid, tile, window_per_head, scale: float, stream=None) -> None:
+    """STA forward on tiled-order [B, heads, L, d] bf16 CUDA tensors."""
+    if q.dim() != 4:
+        raise ValueError("q must be [batch, heads, L, d]")
+    B, Hn, L, d = (int(x) for x in q.shape)
+    for name, t in (("k", k), ("v", v), ("out", out)):
+        if tuple(t.shape) != tuple(q.shape):
+            raise ValueError(f"{name} shape {tuple(t.shape)} differs from q {tuple(q.shape)}")
+    if len(window_per_head) != Hn:
+        raise ValueError("one window per head is required")
+    st = load_library().sta_attention_fwd(_tensor_ptr(q, "q"), _tensor_ptr(k, "k"), _tensor_ptr(v, "v"),
+                                          _tensor_ptr(out, "out"), B, Hn, d, _d3(grid), _d3(tile),
+                                          _windows(window_per_head), float(scale), _stream(stream))
+    _check(st, "sta_attention_fwd")
+
+
+def sta_check_device_status(stream=None) -> int:
+    """Synchronises the stream; returns STA_OK or STA_ERR_TIMEOUT (raises on CUDA errors)."""
+    st = load_library().sta_check_device_status(_stream(stream))
+    if st not in (STA_OK, STA_ERR_TIMEOUT):
+        _check(st, "sta_check_device_status")
+    return st
+
+
+def sta_selftest_bounded_wait(limit_ns: int, stream=None) -> int:
+    st = load_library().sta_selftest_bounded_wait(int(limit_ns), _stream(stream))
+    if st not in (STA_OK, STA_ERR_TIMEOUT):
+        _check(st, "sta_selftest_bounded_wait")
+    return st
+
+
+def sta_shutdown() -> None:
+    load_library().sta_shutdown()
+
+
+def sta_forward(q, k, v, grid, tile, window_per_head, scale: Optional[float] = None,
+                stream=None, workspace: Optional[Tuple] = None):
+    """Full STA forward on raster-order [B, heads, L, d] bf16 CUDA tensors.
+
+    Reorders q, k and v to tiled order, runs the tile-windowed attention and
+    reorders the output back, all on ``stream``.  ``workspace`` may hold four
+    preallocated tensors shaped like q (tiled q, k, v and output); otherwise
+    they are allocated with torch.  Returns the raster-order output.
+    """
+    import torch
+    if scale is None:
+        scale = 1.0 / float(q.shape[-1]) ** 0.5
+    if workspace is None:
+        workspace = tuple(torch.empty_like(q) for _ in range(4))
+    qt, kt, vt, ot = workspace
+    out = torch.empty_like(q)
+    sta_tile_reorder(q, qt, grid, tile, stream)
+    sta_tile_reorder(k, kt, grid, tile, stream)
+    sta_tile_reorder(v, vt, grid, tile, stream)
+    sta_attention_fwd(qt, kt, vt, ot, grid, tile, window_per_head, scale, stream)
+    sta_tile_unorder(ot, out, grid, tile, stream)
+    return out

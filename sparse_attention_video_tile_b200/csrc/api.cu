@@ -1,0 +1,309 @@
+// api.cu - the C ABI declared in include/sta.h: argument validation, the
+// schedule cache, the device status word, and the kernel launches.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstring>
+#include <list>
+#include <map>
+#include <memory>
+#include <mutex>
+#include <string>
+#include <tuple>
+#include <vector>
+
+#include "internal.h"
+
+namespace sta {
+namespace {
+
+thread_local std::string g_last_cuda_error;
+
+sta_status cuda_fail(cudaError_t e) {
+  g_last_cuda_error = cudaGetErrorString(e);
+  return STA_ERR_CUDA;
+}
+
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per bounded wait
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlaps(const void* a, const void* b, int64_t bytes) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + static_cast<uintptr_t>(bytes) && y < x + static_cast<uintptr_t>(bytes);
+}
+
+// Device check: compute capability 10.0 (B200, sm_100a code).
+sta_status check_device(int* dev_out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  int major = 0, minor = 0;
+  if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess) return cuda_fail(e);
+  if ((e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess) return cuda_fail(e);
+  if (major != 10 || minor != 0) return STA_ERR_ARCH;
+  if (dev_out) *dev_out = dev;
+  return STA_OK;
+}
+
+// ---------------------------------------------------------------- per-device state
+
+struct CachedSchedule {
+  HostSchedule host;
+  WorkItem* d_items = nullptr;
+  int32_t* d_kv_rows = nullptr;
+  int16_t* d_head_win = nullptr;
+};
+
+using ScheduleKey = std::tuple<int32_t, int32_t, int32_t, int32_t, int32_t, int32_t, int32_t, int32_t,
+                               std::vector<int32_t>>;
+
+struct DeviceState {
+  int32_t* d_err = nullptr;  // bounded-wait status word
+  std::list<std::pair<ScheduleKey, std::unique_ptr<CachedSchedule>>> schedules;  // most recent first
+};
+
+std::mutex g_mu;
+std::map<int, DeviceState> g_devices;
+constexpr size_t kMaxCachedSchedules = 16;
+
+void free_schedule(CachedSchedule* s) {
+  if (s->d_items) cudaFree(s->d_items);
+  if (s->d_kv_rows) cudaFree(s->d_kv_rows);
+  if (s->d_head_win) cudaFree(s->d_head_win);
+  s->d_items = nullptr;
+  s->d_kv_rows = nullptr;
+  s->d_head_win = nullptr;
+}
+
+// Caller holds g_mu.
+sta_status device_state(int dev, DeviceState** out) {
+  DeviceState& st = g_devices[dev];
+  if (!st.d_err) {
+    cudaError_t e = cudaMalloc(&st.d_err, 256);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if ((e = cudaMemset(st.d_err, 0, 256)) != cudaSuccess) return cuda_fail(e);
+  }
+  *out = &st;
+  return STA_OK;
+}
+
+template <typename T>
+cudaError_t upload(T** dst, const std::vector<T>& v) {
+  const size_t bytes = std::max<size_t>(v.size() * sizeof(T), 16);
+  cudaError_t e = cudaMalloc(dst, bytes);
+  if (e != cudaSuccess) return e;
+  if (!v.empty()) e = cudaMemcpy(*dst, v.data(), v.size() * sizeof(T), cudaMemcpyHostToDevice);
+  return e;
+}
+
+// Caller holds g_mu.
+sta_status get_schedule(DeviceState* st, const Geometry& g, int32_t batch, int32_t heads,
+                        const sta_dim3* windows, CachedSchedule** out) {
+  std::vector<int32_t> wv(static_cast<size_t>(heads) * 3);
+  for (int32_t h = 0; h < heads; ++h) {
+    wv[h * 3 + 0] = windows[h].t;
+    wv[h * 3 + 1] = windows[h].h;
+    wv[h * 3 + 2] = windows[h].w;
+  }
+  ScheduleKey key{batch, heads, g.T, g.H, g.W, g.tt, g.th, g.tw, std::move(wv)};
+  for (auto it = st->schedules.begin(); it != st->schedules.end(); ++it) {
+    if (it->first == key) {
+      st->schedules.splice(st->schedules.begin(), st->schedules, it);
+      *out = st->schedules.front().second.get();
+      return STA_OK;
+    }
+  }
+  auto cs = std::make_unique<CachedSchedule>();
+  build_schedule(g, batch, heads, windows, &cs->host);
+  for (const WorkItem& w : cs->host.items)
+    if (w.kv_len < 1) return STA_ERR_ARG;  // cannot happen: a tile always sees itself
+  cudaError_t e;
+  if ((e = upload(&cs->d_items, cs->host.items)) != cudaSuccess ||
+      (e = upload(&cs->d_kv_rows, cs->host.kv_rows)) != cudaSuccess ||
+      (e = upload(&cs->d_head_win, cs->host.head_win)) != cudaSuccess) {
+    free_schedule(cs.get());
+    return cuda_fail(e);
+  }
+  st->schedules.emplace_front(std::move(key), std::move(cs));
+  while (st->schedules.size() > kMaxCachedSchedules) {
+    free_schedule(st->schedules.back().second.get());
+    st->schedules.pop_back();
+  }
+  *out = st->schedules.front().second.get();
+  return STA_OK;
+}
+
+sta_status validate_tensor_args(const void* src, const void* dst, int64_t batch_heads, int32_t d,
+                                sta_dim3 grid, sta_dim3 tile, Geometry* g) {
+  if (!src || !dst) return STA_ERR_NULL;
+  if (!aligned16(src) || !aligned16(dst)) return STA_ERR_ALIGN;
+  if (d != 64 && d != 128) return STA_ERR_HEADDIM;
+  sta_status s = make_geometry(grid, tile, g);
+  if (s != STA_OK) return s;
+  if (batch_heads < 0 || batch_heads > (int64_t(1) << 31)) return STA_ERR_ARG;
+  const int64_t bytes = batch_heads * g->L * d * 2;
+  if (batch_heads > 0 && overlaps(src, dst, bytes)) return STA_ERR_ALIAS;
+  return STA_OK;
+}
+
+}  // namespace
+}  // namespace sta
+
+using namespace sta;
+
+extern "C" {
+
+const char* sta_status_str(sta_status s) {
+  switch (s) {
+    case STA_OK: return "STA_OK";
+    case STA_ERR_NULL: return "STA_ERR_NULL";
+    case STA_ERR_ALIGN: return "STA_ERR_ALIGN";
+    case STA_ERR_ALIAS: return "STA_ERR_ALIAS";
+    case STA_ERR_SHAPE: return "STA_ERR_SHAPE";
+    case STA_ERR_WINDOW: return "STA_ERR_WINDOW";
+    case STA_ERR_HEADDIM: return "STA_ERR_HEADDIM";
+    case STA_ERR_ARCH: return "STA_ERR_ARCH";
+    case STA_ERR_CUDA: return "STA_ERR_CUDA";
+    case STA_ERR_TIMEOUT: return "STA_ERR_TIMEOUT";
+    case STA_ERR_ARG: return "STA_ERR_ARG";
+  }
+  return "STA_ERR_UNKNOWN";
+}
+
+const char* sta_last_cuda_error(void) { return g_last_cuda_error.c_str(); }
+
+sta_status sta_tile_index_map(sta_dim3 grid, sta_dim3 tile, int32_t* tiled_of_raster) {
+  Geometry g;
+  sta_status s = make_geometry(grid, tile, &g);
+  if (s != STA_OK) return s;
+  if (!tiled_of_raster) return STA_ERR_NULL;
+  // Walk tiles in raster order over the tile grid and tokens in raster order
+  // inside each tile; the running counter is the tiled row.
+  int32_t m = 0;
+  for (int32_t at = 0; at < g.nT; ++at)
+    for (int32_t ah = 0; ah < g.nH; ++ah)
+      for (int32_t aw = 0; aw < g.nW; ++aw)
+        for (int32_t lt = 0; lt < g.tt; ++lt)
+          for (int32_t lh = 0; lh < g.th; ++lh)
+            for (int32_t lw = 0; lw < g.tw; ++lw) {
+              const int64_t n = (static_cast<int64_t>(at * g.tt + lt) * g.H + (ah * g.th + lh)) * g.W + aw * g.tw + lw;
+              tiled_of_raster[n] = m++;
+            }
+  return STA_OK;
+}
+
+int64_t sta_attended_pairs(int32_t batch, int32_t heads, sta_dim3 grid, sta_dim3 tile, const sta_dim3* windows) {
+  Geometry g;
+  if (make_geometry(grid, tile, &g) != STA_OK || batch < 0 || heads < 0 || (heads > 0 && !windows)) return -1;
+  int64_t total = 0;
+  for (int32_t h = 0; h < heads; ++h) {
+    if (windows[h].t < 1 || windows[h].h < 1 || windows[h].w < 1) return -1;
+    const int64_t wt = std::min(windows[h].t, g.nT), wh = std::min(windows[h].h, g.nH), ww = std::min(windows[h].w, g.nW);
+    total += g.L * g.ntile * wt * wh * ww;
+  }
+  return total * batch;
+}
+
+sta_status sta_tile_reorder(const void* src, void* dst, int64_t batch_heads, int32_t d, sta_dim3 grid,
+                            sta_dim3 tile, void* stream) {
+  Geometry g;
+  sta_status s = validate_tensor_args(src, dst, batch_heads, d, grid, tile, &g);
+  if (s != STA_OK) return s;
+  if ((s = check_device(nullptr)) != STA_OK) return s;
+  cudaError_t e = launch_reorder(src, dst, batch_heads, d, g, true, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? STA_OK : cuda_fail(e);
+}
+
+sta_status sta_tile_unorder(const void* src, void* dst, int64_t batch_heads, int32_t d, sta_dim3 grid,
+                            sta_dim3 tile, void* stream) {
+  Geometry g;
+  sta_status s = validate_tensor_args(src, dst, batch_heads, d, grid, tile, &g);
+  if (s != STA_OK) return s;
+  if ((s = check_device(nullptr)) != STA_OK) return s;
+  cudaError_t e = launch_reorder(src, dst, batch_heads, d, g, false, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? STA_OK : cuda_fail(e);
+}
+
+sta_status sta_attention_fwd(const void* q, const void* k, const void* v, void* out, int32_t batch,
+                             int32_t heads, int32_t d, sta_dim3 grid, sta_dim3 tile,
+                             const sta_dim3* window_per_head, float scale, void* stream) {
+  if (!q || !k || !v || !out || !window_per_head) return STA_ERR_NULL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return STA_ERR_ALIGN;
+  if (d != 64 && d != 128) return STA_ERR_HEADDIM;
+  Geometry g;
+  sta_status s = make_geometry(grid, tile, &g);
+  if (s != STA_OK) return s;
+  if (batch < 1 || heads < 1 || static_cast<int64_t>(batch) * heads > (int64_t(1) << 24)) return STA_ERR_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return STA_ERR_ARG;
+  for (int32_t h = 0; h < heads; ++h)
+    if (window_per_head[h].t < 1 || window_per_head[h].h < 1 || window_per_head[h].w < 1) return STA_ERR_WINDOW;
+  const int64_t bytes = static_cast<int64_t>(batch) * heads * g.L * d * 2;
+  if (overlaps(out, q, bytes) || overlaps(out, k, bytes) || overlaps(out, v, bytes)) return STA_ERR_ALIAS;
+  int dev = 0;
+  if ((s = check_device(&dev)) != STA_OK) return s;
+
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState* st = nullptr;
+  if ((s = device_state(dev, &st)) != STA_OK) return s;
+  CachedSchedule* cs = nullptr;
+  if ((s = get_schedule(st, g, batch, heads, window_per_head, &cs)) != STA_OK) return s;
+  DeviceSchedule ds{cs->d_items, cs->d_kv_rows, cs->d_head_win, static_cast<int32_t>(cs->host.items.size()),
+                    cs->host.masked};
+  cudaError_t e = launch_attention(q, k, v, out, batch, heads, d, g, ds, scale, st->d_err, kWaitLimitNs,
+                                   static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? STA_OK : cuda_fail(e);
+}
+
+sta_status sta_check_device_status(void* stream) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if ((e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream))) != cudaSuccess) return cuda_fail(e);
+  std::lock_guard<std::mutex> lock(g_mu);
+  auto it = g_devices.find(dev);
+  if (it == g_devices.end() || !it->second.d_err) return STA_OK;
+  int32_t flag = 0;
+  if ((e = cudaMemcpy(&flag, it->second.d_err, sizeof(flag), cudaMemcpyDeviceToHost)) != cudaSuccess)
+    return cuda_fail(e);
+  if (flag != 0) {
+    if ((e = cudaMemset(it->second.d_err, 0, sizeof(int32_t))) != cudaSuccess) return cuda_fail(e);
+    return STA_ERR_TIMEOUT;
+  }
+  return STA_OK;
+}
+
+sta_status sta_selftest_bounded_wait(uint64_t limit_ns, void* stream) {
+  if (limit_ns < 100000ull) limit_ns = 100000ull;
+  if (limit_ns > 5000000000ull) limit_ns = 5000000000ull;
+  sta_status s;
+  int dev = 0;
+  if ((s = check_device(&dev)) != STA_OK) return s;
+  int32_t* err = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceState* st = nullptr;
+    if ((s = device_state(dev, &st)) != STA_OK) return s;
+    err = st->d_err;
+  }
+  cudaError_t e = launch_selftest_wait(err, limit_ns, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  return sta_check_device_status(stream);
+}
+
+void sta_shutdown(void) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  int cur = 0;
+  cudaGetDevice(&cur);
+  for (auto& kv : g_devices) {
+    if (cudaSetDevice(kv.first) != cudaSuccess) continue;
+    for (auto& s : kv.second.schedules) free_schedule(s.second.get());
+    kv.second.schedules.clear();
+    if (kv.second.d_err) cudaFree(kv.second.d_err);
+    kv.second.d_err = nullptr;
+  }
+  g_devices.clear();
+  cudaSetDevice(cur);
+}
+
+}  // extern "C"

@@ -1,0 +1,102 @@
+"""C-ABI checks that need no GPU: exported symbols, host-only entry points
+against the oracle, and argument validation (which returns before any device
+call).  With valid arguments on a machine without a GPU the product path must
+fail loudly (a CUDA or architecture error), never fall back to the CPU.
+"""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle.sta_oracle as O
+from workloads import CONFIGS
+
+import sparse_attention_video_tile_b200 as sta
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _header_functions():
+    txt = open(os.path.join(ROOT, "include", "sta.h")).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(sta_\w+)\s*\(", txt)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from sparse_attention_video_tile_b200.build import build
+    build()
+    return sta.load_library()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _header_functions()
+    assert len(names) >= 9
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings(lib):
+    for code, name in sta.STATUS_NAMES.items():
+        assert sta.sta_status_str(code) == name
+
+
+@pytest.mark.parametrize("grid,tile", [((2, 2, 4), (1, 2, 2)), ((4, 8, 8), (2, 4, 4)), ((12, 24, 40), (6, 8, 8)),
+                                       ((30, 48, 80), (6, 8, 8)), ((1, 128, 128), (1, 8, 16)),
+                                       ((48, 48, 80), (6, 8, 8)), ((3, 10, 10), (1, 5, 5))])
+def test_index_map_bit_exact_vs_oracle(lib, grid, tile):
+    got = sta.sta_tile_index_map(grid, tile)
+    want = O.tiled_of_raster(grid, tile)
+    assert got.dtype == np.int32
+    assert np.array_equal(got.astype(np.int64), want)
+
+
+@pytest.mark.parametrize("name", sorted(CONFIGS))
+def test_attended_pairs_vs_oracle(lib, name):
+    c = CONFIGS[name]
+    assert sta.sta_attended_pairs(c.batch, c.heads, c.grid, c.tile, c.windows) == \
+        O.attended_pairs(c.batch, c.grid, c.tile, c.windows)
+
+
+def _call_reorder(lib, src, dst, bh=1, d=128, grid=(4, 8, 8), tile=(2, 4, 4)):
+    return lib.sta_tile_reorder(src, dst, bh, d, sta._d3(grid), sta._d3(tile), None)
+
+
+def _call_attn(lib, q=0x10000, k=0x20000, v=0x30000, out=0x40000, batch=1, heads=2, d=64,
+               grid=(4, 8, 8), tile=(2, 4, 4), windows=((1, 1, 1), (3, 3, 3)), scale=0.125):
+    return lib.sta_attention_fwd(q, k, v, out, batch, heads, d, sta._d3(grid), sta._d3(tile),
+                                 sta._windows(windows), ctypes.c_float(scale), None)
+
+
+def test_validation_codes(lib):
+    A, B = 0x100000, 0x200000   # fake, never dereferenced: validation fails first
+    assert _call_reorder(lib, None, B) == 1
+    assert _call_reorder(lib, A + 2, B) == 2
+    assert _call_reorder(lib, A, A) == 3
+    assert _call_reorder(lib, A, A + 1024) == 3                      # overlapping ranges
+    assert _call_reorder(lib, A, B, grid=(4, 8, 9)) == 4
+    assert _call_reorder(lib, A, B, grid=(0, 8, 8)) == 4
+    assert _call_reorder(lib, A, B, d=96) == 6
+    assert lib.sta_tile_unorder(A, B, 1, 128, sta._d3((4, 8, 9)), sta._d3((2, 4, 4)), None) == 4
+    assert _call_attn(lib, q=None) == 1
+    assert _call_attn(lib, out=0x40008) == 2
+    assert _call_attn(lib, out=0x10000) == 3
+    assert _call_attn(lib, d=80) == 6
+    assert _call_attn(lib, tile=(3, 4, 4)) == 4
+    assert _call_attn(lib, windows=((1, 0, 1), (3, 3, 3))) == 5
+    assert _call_attn(lib, scale=0.0) == 10
+    assert _call_attn(lib, scale=float("nan")) == 10
+    assert _call_attn(lib, batch=0) == 10
+    assert lib.sta_tile_index_map(sta._d3((4, 8, 8)), sta._d3((2, 4, 4)), None) == 1
+    assert lib.sta_attended_pairs(1, 1, sta._d3((4, 8, 8)), sta._d3((3, 4, 4)), sta._windows([(1, 1, 1)])) == -1
+
+
+def test_no_cpu_fallback_without_gpu(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    # valid arguments: the library must report a CUDA/architecture error, not compute on the host
+    assert _call_reorder(lib, 0x100000, 0x200000) in (7, 8)
+    assert _call_attn(lib) in (7, 8)
