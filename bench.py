@@ -1,0 +1,356 @@
+"""Benchmark of the Sliding Tile Attention forward path on B200.
+
+One step = the whole hot path on one batch of synthetic input: reorder q, k
+and v to tiled order, tile-windowed attention, reorder the output back.  The
+default workload is the HunyuanVideo-shaped one (latent 30x48x80 = 115200
+tokens, tile (6,8,8), window (3,3,3) tiles, 24 heads, d = 128, bf16).
+
+value = attended FLOPs (4 * d * attended query-key pairs) of all ranks per
+second of step time, device-timed with CUDA events (max over ranks).  Inputs
+(708 MB per tensor) are larger than L2, so no flush is needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With --impl reference the CPU oracle is timed instead (rank 0 only).
+Multi-GPU runs are independent replicas: the path has no exchange step.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "STA fwd ms & TFLOPS (attended) at 30×48×80, 24 heads, d=128; % of BF16 peak"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        d["_source"] = "measured"
+        return d
+    d = dict(PEAKS_FALLBACK)
+    d["_source"] = "fallback"
+    return d
+
+
+# ---------------------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        loaded = [s for s in sm if s > 0.5 * (max(sm) if sm else 1)]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in rows:
+            for i, n in enumerate(names):
+                if r[5 + i].lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------- reference (CPU oracle) arm
+
+
+def oracle_sample_tflops(cfg, n_rows: int, head: int, seed: int = 0):
+    """Times the CPU oracle on `n_rows` query rows of one head; returns
+    (attended TFLOP/s, seconds, rows)."""
+    import numpy as np
+    import oracle.sta_oracle as O
+    import workloads as W
+    q, k, v = W.make_head(cfg, seed, 0, head)
+    q, k, v = (x.double().numpy() for x in (q, k, v))
+    rng = np.random.default_rng(seed + head)
+    rows = np.sort(rng.choice(cfg.L, size=n_rows, replace=False))
+    w = cfg.windows[head]
+    pairs_per_row = O.attended_pairs_head(cfg.grid, cfg.tile, w) // cfg.L
+    t0 = time.perf_counter()
+    O.sta_attention_head(q, k, v, cfg.grid, cfg.tile, w, cfg.scale, rows=rows)
+    dt = time.perf_counter() - t0
+    return 4.0 * cfg.d * pairs_per_row * n_rows / dt / 1e12, dt, n_rows
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def run_reference(args, cfg):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    rows = args.ref_rows
+    for i in range(args.warmup):
+        oracle_sample_tflops(cfg, rows, head=i % cfg.heads, seed=i)
+    vals, secs = [], []
+    for i in range(args.steps):
+        tf, dt, _ = oracle_sample_tflops(cfg, rows, head=i % cfg.heads, seed=100 + i)
+        vals.append(tf)
+        secs.append(dt)
+    value = statistics.median(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * statistics.median(secs),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_dict(cfg, args),
+        "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"{rows} random query rows of one head per step (explicit-mask fp64 "
+                                   f"attention over all {cfg.L} keys); heads cycle over steps"},
+        "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------- our arm
+
+
+def config_dict(cfg, args):
+    win = sorted(set(cfg.windows))
+    return {"workload": f"{cfg.name}: B={cfg.batch}, heads={cfg.heads}, d={cfg.d}, grid={cfg.grid}, "
+                        f"tile={cfg.tile}, window={win[0] if len(win) == 1 else 'per head'}",
+            "batch": cfg.batch, "heads": cfg.heads, "d": cfg.d, "grid": list(cfg.grid), "tile": list(cfg.tile),
+            "windows": [list(w) for w in win], "seq_len": cfg.L,
+            "l2": "inputs larger than L2 (%.0f MB per tensor), no flush" % (cfg.batch * cfg.heads * cfg.L * cfg.d * 2 / 1e6),
+            "parallelism": f"replicas x{args.gpus}"}
+
+
+def run_ours(args, cfg):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import sparse_attention_video_tile_b200 as sta
+    import workloads as W
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+
+    sta.load_library()
+    peaks = load_peaks()
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+
+    q_h, k_h, v_h = (x.pin_memory() for x in W.make_qkv(cfg, seed=rank))
+    q, k, v = (x.to(dev, non_blocking=True) for x in (q_h, k_h, v_h))
+    ws = [torch.empty_like(q) for _ in range(4)]  # tiled q, k, v, out
+    out = torch.empty_like(q)
+    out_h = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+    qt, kt, vt, ot = ws
+    grid, tile, wins, scale = cfg.grid, cfg.tile, cfg.windows, cfg.scale
+    flops = 4.0 * cfg.d * sta.sta_attended_pairs(cfg.batch, cfg.heads, grid, tile, wins)
+    tensor_bytes = q.numel() * q.element_size()
+
+    ev = {n: [] for n in ("r0", "r1", "a0", "a1", "u0", "u1")}
+
+    def step(record: bool):
+        if record:
+            e = {n: torch.cuda.Event(enable_timing=True) for n in ev}
+            e["r0"].record(stream)
+        sta.sta_tile_reorder(q, qt, grid, tile, stream)
+        sta.sta_tile_reorder(k, kt, grid, tile, stream)
+        sta.sta_tile_reorder(v, vt, grid, tile, stream)
+        if record:
+            e["r1"].record(stream)
+            e["a0"].record(stream)
+        sta.sta_attention_fwd(qt, kt, vt, ot, grid, tile, wins, scale, stream)
+        if record:
+            e["a1"].record(stream)
+            e["u0"].record(stream)
+        sta.sta_tile_unorder(ot, out, grid, tile, stream)
+        if record:
+            e["u1"].record(stream)
+            for n in ev:
+                ev[n].append(e[n])
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+
+    for _ in range(args.warmup):
+        step(False)
+    if sta.sta_check_device_status(stream) != sta.STA_OK:
+        raise RuntimeError("a kernel gave up on a bounded wait during warm-up")
+
+    # ---- device-resident timing
+    barrier()
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        time.sleep(1.0)  # nvidia-smi needs a moment before its first sample
+        t_start.record(stream)
+        for _ in range(args.steps):
+            step(True)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    ms_total = t_start.elapsed_time(t_end)
+    if world > 1:
+        tt = torch.tensor([ms_total], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_total = float(tt.item())
+    ms_step = ms_total / args.steps
+    value = world * flops / (ms_step * 1e-3) / 1e12
+    att_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(ev["a0"], ev["a1"]))
+    reo_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(ev["r0"], ev["r1"])) / 3.0
+    uno_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(ev["u0"], ev["u1"]))
+    if sta.sta_check_device_status(stream) != sta.STA_OK:
+        raise RuntimeError("a kernel gave up on a bounded wait during timing")
+
+    # ---- end to end through the public API with host buffers
+    e2e_steps = max(1, min(args.steps, args.e2e_steps))
+    barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        q.copy_(q_h, non_blocking=True)
+        k.copy_(k_h, non_blocking=True)
+        v.copy_(v_h, non_blocking=True)
+        o = sta.sta_forward(q, k, v, grid, tile, wins, scale, stream, workspace=ws)
+        out_h.copy_(o, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if world > 1:
+        tt = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+
+    peak_s = peaks.get("bf16_tflops_sustained", PEAKS_FALLBACK["bf16_tflops_sustained"])
+    peak_b = peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"])
+    hbm = peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"])
+    att_tflops = flops / (att_ms * 1e-3) / 1e12
+    reo_gbs = 2 * tensor_bytes / (reo_ms * 1e-3) / 1e9
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tf, dt, rows = oracle_sample_tflops(cfg, args.cpu_rows, head=0)
+        cpu = {"value": tf, "unit": "TFLOPS", "cores": blas_threads(), "kind": "oracle",
+               "sample": f"{rows} random query rows of head 0 ({dt:.1f} s): explicit-mask fp64 attention "
+                         f"over all {cfg.L} keys, attended FLOPs only"}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(cfg, args),
+        "roofline": {"bound": "tensor", "kernel": "sta_fwd_kernel", "achieved": att_tflops, "peak": peak_s,
+                     "unit": "TFLOP/s", "frac": att_tflops / peak_s, "traffic": None,
+                     "peak_kind": f"bf16_tflops_sustained ({peaks['_source']})",
+                     "frac_of_burst_peak": att_tflops / peak_b, "frac_of_2250_datasheet": att_tflops / 2250.0},
+        "kernels": {"attention_ms": att_ms, "attention_tflops": att_tflops,
+                    "reorder_ms_per_tensor": reo_ms, "reorder_gbs": reo_gbs, "reorder_frac_hbm": reo_gbs / hbm,
+                    "unorder_ms": uno_ms, "unorder_gbs": 2 * tensor_bytes / (uno_ms * 1e-3) / 1e9},
+        "cpu_baseline": cpu,
+        "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS", "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": 3 * tensor_bytes, "d2h_bytes_per_step": tensor_bytes,
+                "steps": e2e_steps},
+        "clocks": clk.summary(),
+        "gpu_launches": 5 * args.steps,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="hunyuan")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--cpu-rows", type=int, default=4096)
+    ap.add_argument("--ref-rows", type=int, default=512)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="use only the first N heads of the workload (small profiling cases)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("at least 3 warm-up steps are required")
+    import workloads as W
+    cfg = W.CONFIGS[args.config]
+    if args.heads:
+        cfg = W.custom_config(f"{cfg.name}[{args.heads} heads]", cfg.batch, args.heads, cfg.d, cfg.grid, cfg.tile,
+                              cfg.windows[:args.heads])
+    if args.impl == "reference":
+        return run_reference(args, cfg)
+    return run_ours(args, cfg)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

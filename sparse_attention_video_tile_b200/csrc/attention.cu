@@ -437,17 +437,19 @@ cudaError_t launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
                      cudaStream_t stream) {
   auto kern = sta_fwd_kernel<D, MASKED>;
   const int smem = Smem<D>::kDynBytes;
-  static bool configured[2] = {false, false};
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  (void)configured;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+  if (e != cudaSuccess) return e;
   int dev = 0, sms = 0, per_sm = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
   if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem)) != cudaSuccess) return e;
   if (per_sm < 1) return cudaErrorInvalidConfiguration;
-  if (per_sm > 2) per_sm = 2;  // TMEM: 256 columns per CTA, 512 per SM
-  int grid = sms * per_sm;
+  // Two CTAs per SM by design (registers, shared memory and TMEM - 2 x 256 of 512
+  // columns - all allow exactly two).  CTAs share nothing, so a grid larger than
+  // what is resident only queues.
+  int grid = sms * 2;
   if (grid > p.n_items) grid = p.n_items;
   if (grid < 1) return cudaSuccess;
   kern<<<grid, kThreads, smem, stream>>>(tq, tk, tv, p);
