@@ -35,6 +35,7 @@
 
 #include <cmath>
 #include <cstdio>
+#include <cstdlib>
 #include <mutex>
 
 #include "internal.h"
@@ -51,6 +52,14 @@ constexpr int kTmemCols = 256;      // S: [0,128), O: [128, 128 + d)
 constexpr int kSCol = 0;
 constexpr int kOCol = 128;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// Register split: launched at 128 per thread (256 threads, two CTAs per SM);
+// the softmax warpgroup takes 208, the other warpgroup keeps 48:
+// 128 * 208 + 128 * 48 = 256 * 128.
+constexpr int kLaunchRegs = 128;
+constexpr int kDefaultPoly16 = 0;
+constexpr int kRegsSoftmax = 208;
+constexpr int kRegsOther = 48;
+static_assert(128 * kRegsSoftmax + 128 * kRegsOther == kThreads * kLaunchRegs, "register split must match the launch");
 
 struct FwdParams {
   const WorkItem* items;
@@ -104,7 +113,7 @@ __device__ __forceinline__ uint64_t vmn_desc(uint32_t base, int k16) {
   return sdesc_sw128(addr, kBlockRows * 128, 1024);
 }
 
-template <int D, bool MASKED>
+template <int D, bool MASKED, int POLY16>
 __global__ void __launch_bounds__(kThreads, 2)
     sta_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -148,6 +157,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 
   if (warp == 4) {
     // ------------------------------------------------------------ producer
+    setmaxnreg_dec<kRegsOther>();
     if (lane == 0) {
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_k);
@@ -190,6 +200,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     __syncwarp();
   } else if (warp == 5) {
     // ------------------------------------------------------------ MMA issuer
+    setmaxnreg_dec<kRegsOther>();
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
@@ -241,8 +252,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     __syncwarp();
   } else if (warp < 4) {
     // ------------------------------------------------------------ softmax + epilogue
+    setmaxnreg_inc<kRegsSoftmax>();
     const int row = threadIdx.x;                          // 0..127 = TMEM lane
     const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const float sl2 = p.scale_log2;
     uint32_t sphase = 0, it = 0;
     bool ok = true;
     for (int w = blockIdx.x; w < p.n_items && ok; w += gridDim.x, ++it) {
@@ -266,31 +279,39 @@ __global__ void __launch_bounds__(kThreads, 2)
         ++sphase;
         if (!ok) break;
         tc_fence_after();
-        const int32_t kv_row = MASKED ? p.kv_rows[item.kv_off + j] : 0;
-        // pass 1: row max of the raw scores
-        float mx = -INFINITY;
+        // The whole score row (128 fp32) in one round trip.
+        uint32_t r[128];
+        tmem_ld32_at<0>(trow + kSCol, r);
+        tmem_ld32_at<32>(trow + kSCol + 32, r);
+        tmem_ld32_at<64>(trow + kSCol + 64, r);
+        tmem_ld32_at<96>(trow + kSCol + 96, r);
+        tmem_wait_ld();
+        if (MASKED) {
+          const int32_t kv_row = p.kv_rows[item.kv_off + j];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t r[32];
-          tmem_ld32(trow + kSCol + c * 32, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            float s = __uint_as_float(r[i]);
-            if (MASKED) {
-              const int32_t key = kv_row + c * 32 + i;
-              bool in = key < p.L;
-              if (in) {
-                const int32_t kt = key / p.ntile;
-                const int32_t bt = kt / (p.nH * p.nW), bh_ = (kt / p.nW) % p.nH, bw = kt % p.nW;
-                in = bt >= ws_t && bt < we_t && bh_ >= ws_h && bh_ < we_h && bw >= ws_w && bw < we_w;
-              }
-              if (!in) s = -INFINITY;
+          for (int i = 0; i < 128; ++i) {
+            const int32_t key = kv_row + i;
+            bool in = key < p.L;
+            if (in) {
+              const int32_t kt = key / p.ntile;
+              const int32_t bt = kt / (p.nH * p.nW), bh_ = (kt / p.nW) % p.nH, bw = kt % p.nW;
+              in = bt >= ws_t && bt < we_t && bh_ >= ws_h && bh_ < we_h && bw >= ws_w && bw < we_w;
             }
-            mx = fmaxf(mx, s);
+            if (!in) r[i] = __float_as_uint(-INFINITY);
           }
         }
-        const float m_blk = mx * p.scale_log2;
+#define SV(i) __uint_as_float(r[i])
+        // Row max: eight independent chains of three-input maxima.
+        float mx8[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          float a = max3f(SV(k), SV(k + 8), SV(k + 16));
+#pragma unroll
+          for (int t = 24; t < 120; t += 16) a = max3f(a, SV(k + t), SV(k + t + 8));
+          mx8[k] = fmaxf(a, SV(k + 120));
+        }
+        const float mx = max3f(max3f(mx8[0], mx8[1], mx8[2]), max3f(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
+        const float m_blk = mx * sl2;
         // The running max moves only when it grows by more than 2^8: p stays <= 256
         // and O and the row sum always carry the same factor, so O / l is exact.
         const bool need = (m_run != -INFINITY) && (m_blk > m_run + kRescaleThreshold);
@@ -308,45 +329,35 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (__any_sync(0xffffffffu, need)) {
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
-            uint32_t r[32];
-            tmem_ld32(trow + kOCol + c * 32, r);
+            uint32_t o[32];
+            tmem_ld32(trow + kOCol + c * 32, o);
             tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * f);
-            tmem_st32(trow + kOCol + c * 32, r);
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
+            tmem_st32(trow + kOCol + c * 32, o);
           }
         }
-        const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-        // pass 2: p = 2^(s * scale * log2e - m), row sum, P (bf16) over S's first 64 columns
+        const float nm = (m_run == -INFINITY) ? 0.f : -m_run;
+        // p = 2^(s * scale * log2e - m): POLY16 of every 16 columns on the FMA pipe,
+        // the rest on MUFU; eight partial row sums; P packed to bf16 pairs.
+        float ls[8];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t r[32];
-          tmem_ld32(trow + kSCol + c * 32, r);
-          tmem_wait_ld();
-          uint32_t pk[16];
+        for (int k = 0; k < 8; ++k) ls[k] = 0.f;
+        uint32_t pk[64];
 #pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            float s0 = __uint_as_float(r[i]), s1 = __uint_as_float(r[i + 1]);
-            if (MASKED) {
-#pragma unroll
-              for (int u = 0; u < 2; ++u) {
-                const int32_t key = kv_row + c * 32 + i + u;
-                bool in = key < p.L;
-                if (in) {
-                  const int32_t kt = key / p.ntile;
-                  const int32_t bt = kt / (p.nH * p.nW), bh_ = (kt / p.nW) % p.nH, bw = kt % p.nW;
-                  in = bt >= ws_t && bt < we_t && bh_ >= ws_h && bh_ < we_h && bw >= ws_w && bw < we_w;
-                }
-                if (!in) { if (u == 0) s0 = -INFINITY; else s1 = -INFINITY; }
-              }
-            }
-            const float p0 = ex2_approx(fmaf(s0, p.scale_log2, -m_use));
-            const float p1 = ex2_approx(fmaf(s1, p.scale_log2, -m_use));
-            l_run += p0 + p1;
-            pk[i / 2] = pack_bf16x2(p0, p1);
-          }
-          tmem_st16(trow + kSCol + c * 16, pk);
+        for (int i = 0; i < 128; i += 2) {
+          const float x0 = fmaf(SV(i), sl2, nm);
+          const float x1 = fmaf(SV(i + 1), sl2, nm);
+          const float p0 = (!MASKED && (i & 15) >= 16 - POLY16) ? exp2_poly3(x0) : ex2_approx(x0);
+          const float p1 = (!MASKED && ((i + 1) & 15) >= 16 - POLY16) ? exp2_poly3(x1) : ex2_approx(x1);
+          ls[i & 7] += p0;
+          ls[(i + 1) & 7] += p1;
+          pk[i >> 1] = pack_bf16x2(p0, p1);
         }
+#undef SV
+        tmem_st32_at<0>(trow + kSCol, pk);
+        tmem_st32_at<32>(trow + kSCol + 32, pk);
+        l_run += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(sb + S::kPFull);
@@ -356,29 +367,33 @@ __global__ void __launch_bounds__(kThreads, 2)
       ok = __all_sync(0xffffffffu, mbar_wait(sb + S::kOFull, it & 1, wc, 8));
       if (!ok) break;
       tc_fence_after();
+      uint32_t o[D];
+      tmem_ld32_at<0>(trow + kOCol, o);
+      tmem_ld32_at<32>(trow + kOCol + 32, o);
+      if constexpr (D == 128) {
+        tmem_ld32_at<64>(trow + kOCol + 64, o);
+        tmem_ld32_at<96>(trow + kOCol + 96, o);
+      }
+      tmem_wait_ld();
+      tc_fence_before();
       const float inv_l = 1.0f / l_run;
       const int32_t qrow = item.q_row0 + row;
-      __nv_bfloat16* orow = p.out + (static_cast<int64_t>(item.bh) * p.L + qrow) * D;
+      if (qrow < p.L) {
+        uint4* dst = reinterpret_cast<uint4*>(p.out + (static_cast<int64_t>(item.bh) * p.L + qrow) * D);
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(trow + kOCol + c * 32, r);
-        tmem_wait_ld();
-        uint4 v4[4];
-        uint32_t* pw = reinterpret_cast<uint32_t*>(v4);
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-          pw[i] = pack_bf16x2(__uint_as_float(r[2 * i]) * inv_l, __uint_as_float(r[2 * i + 1]) * inv_l);
-        if (qrow < p.L) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) dst[i] = v4[i];
+        for (int c = 0; c < D / 8; ++c) {
+          uint4 v4;
+          v4.x = pack_bf16x2(__uint_as_float(o[8 * c + 0]) * inv_l, __uint_as_float(o[8 * c + 1]) * inv_l);
+          v4.y = pack_bf16x2(__uint_as_float(o[8 * c + 2]) * inv_l, __uint_as_float(o[8 * c + 3]) * inv_l);
+          v4.z = pack_bf16x2(__uint_as_float(o[8 * c + 4]) * inv_l, __uint_as_float(o[8 * c + 5]) * inv_l);
+          v4.w = pack_bf16x2(__uint_as_float(o[8 * c + 6]) * inv_l, __uint_as_float(o[8 * c + 7]) * inv_l);
+          dst[c] = v4;
         }
       }
-      tc_fence_before();
     }
+  } else {
+    setmaxnreg_dec<kRegsOther>();  // warps 6-7: no role
   }
-  // warps 6-7 have no role.
 
   tc_fence_before();
   __syncthreads();
@@ -432,15 +447,20 @@ bool make_tmap(CUtensorMap* m, const void* base, int64_t bh, int64_t L, int d) {
   return r == CUDA_SUCCESS;
 }
 
-template <int D, bool MASKED>
+template <int D, bool MASKED, int POLY16>
 cudaError_t launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
                      cudaStream_t stream) {
-  auto kern = sta_fwd_kernel<D, MASKED>;
+  auto kern = sta_fwd_kernel<D, MASKED, POLY16>;
   const int smem = Smem<D>::kDynBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) return e;
+  // setmaxnreg redistributes the registers a CTA is launched with; the split in
+  // the kernel adds up only if the kernel was compiled to exactly kLaunchRegs.
+  cudaFuncAttributes fa;
+  if ((e = cudaFuncGetAttributes(&fa, kern)) != cudaSuccess) return e;
+  if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
   int dev = 0, sms = 0, per_sm = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
@@ -454,6 +474,32 @@ cudaError_t launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
   if (grid < 1) return cudaSuccess;
   kern<<<grid, kThreads, smem, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
+}
+
+// Share of exponentials computed on the FMA pipe, in sixteenths (the rest use
+// MUFU ex2).  STA_EXP_POLY16 in the environment overrides the default; only the
+// instantiated values are accepted.
+int exp_poly16() {
+  static int v = [] {
+    const char* e = std::getenv("STA_EXP_POLY16");
+    int x = e ? std::atoi(e) : kDefaultPoly16;
+    if (x != 0 && x != 4 && x != 6 && x != 8) x = kDefaultPoly16;
+    return x;
+  }();
+  return v;
+}
+
+template <int D, bool MASKED>
+cudaError_t launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
+                     cudaStream_t stream) {
+  if (MASKED) return launch_t<D, MASKED, 0>(tq, tk, tv, p, stream);
+  switch (exp_poly16()) {
+    case 0: return launch_t<D, MASKED, 0>(tq, tk, tv, p, stream);
+    case 4: return launch_t<D, MASKED, 4>(tq, tk, tv, p, stream);
+    case 8: return launch_t<D, MASKED, 8>(tq, tk, tv, p, stream);
+    case 6: return launch_t<D, MASKED, 6>(tq, tk, tv, p, stream);
+    default: return launch_t<D, MASKED, 0>(tq, tk, tv, p, stream);
+  }
 }
 
 }  // namespace
@@ -479,9 +525,9 @@ cudaError_t launch_attention(const void* q, const void* k, const void* v, void* 
   p.err = err_flag;
   p.limit_ns = limit_ns;
   if (d == 128) {
-    return s.masked ? launch_t<128, true>(tq, tk, tv, p, stream) : launch_t<128, false>(tq, tk, tv, p, stream);
+    return s.masked ? launch_d<128, true>(tq, tk, tv, p, stream) : launch_d<128, false>(tq, tk, tv, p, stream);
   }
-  return s.masked ? launch_t<64, true>(tq, tk, tv, p, stream) : launch_t<64, false>(tq, tk, tv, p, stream);
+  return s.masked ? launch_d<64, true>(tq, tk, tv, p, stream) : launch_d<64, false>(tq, tk, tv, p, stream);
 }
 
 cudaError_t launch_selftest_wait(int32_t* err_flag, uint64_t limit_ns, cudaStream_t stream) {
