@@ -6,28 +6,32 @@
 // innovation"), and the kernel is built around asynchronous loads and block
 // management (summary page, "AI overview").  On B200 that becomes:
 //
-//   * one CTA works on a block of 128 query rows at a time (persistent grid,
-//     two CTAs per SM, work items from the host window enumerator);
-//   * warp 4, the producer, streams Q once per item and then only the key and
-//     value blocks of the window into a two-stage shared-memory ring with TMA
-//     (128-byte swizzle, completion on mbarriers);
-//   * warp 5 issues tcgen05 MMAs from one thread: S = Q K^T (both operands in
-//     shared memory, fp32 accumulator in TMEM columns [0, 128)) and O += P V
-//     (P read from TMEM where it overwrote S, V from shared memory, O in TMEM
-//     columns [128, 128 + d));
-//   * warps 0-3 (128 threads, one query row each, TMEM lane = row) run the
-//     online softmax in fp32: row max, p = 2^(s*scale*log2e - m), row sum,
-//     P rounded to bf16 and written back to TMEM; O is rescaled only when the
-//     running max grows by more than 2^8 (the result is unchanged: O and the
-//     row sum always carry the same factor), then the epilogue divides by the
+//   * a persistent grid of one CTA per SM; each CTA runs two lanes, each lane a
+//     block of 128 query rows (one work item of the host window enumerator) at a
+//     time;
+//   * warp 8, the producer, streams each lane's Q once per item and then only
+//     the key and value blocks of the lane's window into a four-stage shared
+//     memory ring with TMA (128-byte swizzle, completion on mbarriers);
+//   * warp 9 issues every tcgen05 MMA from one thread: S = Q K^T (both operands
+//     in shared memory, fp32 accumulator in TMEM) and O += P V (P read from TMEM
+//     where it overwrote S, V from shared memory, O in TMEM);
+//   * warps 0-3 (lane 0) and 4-7 (lane 1), one query row per thread, TMEM lane
+//     = row, run the online softmax in fp32: row max, p = 2^(s*scale*log2e - m),
+//     row sum, P rounded to bf16 and written back to TMEM; O is rescaled only
+//     when the running max grows by more than 2^8 (the result is unchanged: O
+//     and the row sum always carry the same factor); the epilogue divides by the
 //     row sum and writes bf16 rows.
+//
+// The producer and the MMA issuer walk the same fixed sequence of turns,
+// alternating lanes: a turn issues a lane's P*V for block j and its Q*K^T for
+// block j+1.  The tensor core therefore always has the other lane's work queued
+// while one lane's softmax runs (ping-pong), and the load order equals the
+// consumption order, so one ring serves both lanes.
+//
 // With Ntile a multiple of 128 no element mask exists at all.  Otherwise
 // (small tiles, ragged tails) the softmax masks whole key tiles outside the
-// row's window and keys past L.
-//
-// The two CTAs on an SM interleave: while one runs its softmax the other's
-// MMAs keep the tensor core busy.  Every wait is bounded (see ptx.cuh): a
-// stuck pipeline records an error code and the CTA drains and exits.
+// row's window and keys past L.  Every wait is bounded (see ptx.cuh): a stuck
+// pipeline records an error code and the CTA drains and exits.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -46,20 +50,22 @@ namespace {
 
 using namespace ptx;
 
-constexpr int kThreads = 256;       // warps 0-3 softmax, 4 producer, 5 MMA, 6-7 idle
-constexpr int kStages = 2;          // key/value ring stages (K and V alternate)
-constexpr int kTmemCols = 256;      // S: [0,128), O: [128, 128 + d)
-constexpr int kSCol = 0;
-constexpr int kOCol = 128;
+constexpr int kLanes = 2;
+constexpr int kThreads = 384;       // warps 0-3 / 4-7 softmax of lane 0 / 1, 8 producer, 9 MMA, 10-11 idle
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kStages = 4;          // key/value ring stages (K and V blocks in consumption order)
+constexpr int kTmemCols = 512;      // lane l: S at 256 l, O at 256 l + 128
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
-// Register split: launched at 128 per thread (256 threads, two CTAs per SM);
-// the softmax warpgroup takes 208, the other warpgroup keeps 48:
-// 128 * 208 + 128 * 48 = 256 * 128.
-constexpr int kLaunchRegs = 128;
-constexpr int kDefaultPoly16 = 0;
+// Register split: launched at 168 per thread (384 threads, one CTA per SM);
+// the two softmax warpgroups take 208 each, the producer/MMA warpgroup keeps 88:
+// 2 * 128 * 208 + 128 * 88 = 384 * 168.
+constexpr int kLaunchRegs = 168;
 constexpr int kRegsSoftmax = 208;
-constexpr int kRegsOther = 48;
-static_assert(128 * kRegsSoftmax + 128 * kRegsOther == kThreads * kLaunchRegs, "register split must match the launch");
+constexpr int kRegsOther = 88;
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsOther == kThreads * kLaunchRegs,
+              "register split must match the launch");
+constexpr int kDefaultPoly16 = 0;
 
 struct FwdParams {
   const WorkItem* items;
@@ -79,25 +85,52 @@ struct FwdParams {
 template <int D>
 struct Smem {
   static constexpr int kBlockBytes = kBlockRows * D * 2;  // one 128-row block of Q, K or V
-  static constexpr int kQ = 0;
-  static constexpr int kStage0 = kBlockBytes;
+  static constexpr int kQ0 = 0;                            // lane l's Q at kQ0 + l * kBlockBytes
+  static constexpr int kStage0 = kLanes * kBlockBytes;
   static constexpr int kBar = kStage0 + kStages * kBlockBytes;
   // barriers (8 bytes each)
-  static constexpr int kQFull = kBar + 0;
-  static constexpr int kQEmpty = kBar + 8;
-  static constexpr int kKvFull = kBar + 16;                 // kStages
-  static constexpr int kKvEmpty = kKvFull + 8 * kStages;    // kStages
-  static constexpr int kSFull = kKvEmpty + 8 * kStages;
-  static constexpr int kPFull = kSFull + 8;
-  static constexpr int kOFull = kPFull + 8;
-  static constexpr int kDrain = kOFull + 8;
+  static constexpr int kQFull = kBar;                      // [lane]
+  static constexpr int kQEmpty = kQFull + 8 * kLanes;      // [lane]
+  static constexpr int kKvFull = kQEmpty + 8 * kLanes;     // [stage]
+  static constexpr int kKvEmpty = kKvFull + 8 * kStages;   // [stage]
+  static constexpr int kSFull = kKvEmpty + 8 * kStages;    // [lane]
+  static constexpr int kPFull = kSFull + 8 * kLanes;       // [lane]
+  static constexpr int kOFull = kPFull + 8 * kLanes;       // [lane]
+  static constexpr int kDrain = kOFull + 8 * kLanes;
   static constexpr int kTmemSlot = kDrain + 8;
   static constexpr int kAbort = kTmemSlot + 4;
   static constexpr int kEnd = kAbort + 4;
-  // + slack to align the base to 1024; never below 96 KB so that at most two CTAs
-  // (2 x 256 TMEM columns) share an SM, whatever d is.
-  static constexpr int kDynBytes = (kEnd + 1024) > 98304 ? (kEnd + 1024) : 98304;
+  static constexpr int kDynBytes = kEnd + 1024;  // + slack to align the base to 1024
+  static_assert(kDynBytes <= 227 * 1024, "shared memory budget");
 };
+
+// Work-item cursor of one lane, shared logic of the producer and the MMA issuer.
+// Lane l of CTA c takes items (k * gridDim.x + c) * 2 + l for k = 0, 1, ...: at
+// any time the CTAs work on adjacent items (neighbouring query blocks).
+struct LaneCursor {
+  int32_t k;        // how many items this lane has finished
+  int32_t idx;      // current item, or -1 when the lane is done
+  int32_t n;        // key blocks of the current item
+  int32_t j;        // next P*V block
+  int32_t kv_off, bh, q_row0;
+  bool started;     // Q*K^T of block 0 issued
+};
+
+__device__ __forceinline__ void cursor_load(LaneCursor& c, const WorkItem* items, int32_t n_items, int lane) {
+  const int32_t idx = (c.k * static_cast<int32_t>(gridDim.x) + static_cast<int32_t>(blockIdx.x)) * kLanes + lane;
+  c.started = false;
+  c.j = 0;
+  if (idx < n_items) {
+    const WorkItem w = items[idx];
+    c.idx = idx;
+    c.n = w.kv_len;
+    c.kv_off = w.kv_off;
+    c.bh = w.bh;
+    c.q_row0 = w.q_row0;
+  } else {
+    c.idx = -1;
+  }
+}
 
 // Descriptor of a K-major bf16 operand stored as [rows][64] boxes of 128 bytes per
 // row (128-byte swizzle); k16 selects the 16-element slice along K.
@@ -114,7 +147,7 @@ __device__ __forceinline__ uint64_t vmn_desc(uint32_t base, int k16) {
 }
 
 template <int D, bool MASKED, int POLY16>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, 1)
     sta_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
   using S = Smem<D>;
@@ -128,20 +161,22 @@ __global__ void __launch_bounds__(kThreads, 2)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::kTmemSlot);
 
   if (threadIdx.x == 0) {
-    mbar_init(sb + S::kQFull, 1);
-    mbar_init(sb + S::kQEmpty, 1);
+    for (int l = 0; l < kLanes; ++l) {
+      mbar_init(sb + S::kQFull + 8 * l, 1);
+      mbar_init(sb + S::kQEmpty + 8 * l, 1);
+      mbar_init(sb + S::kSFull + 8 * l, 1);
+      mbar_init(sb + S::kPFull + 8 * l, 128);
+      mbar_init(sb + S::kOFull + 8 * l, 1);
+    }
     for (int s = 0; s < kStages; ++s) {
       mbar_init(sb + S::kKvFull + 8 * s, 1);
       mbar_init(sb + S::kKvEmpty + 8 * s, 1);
     }
-    mbar_init(sb + S::kSFull, 1);
-    mbar_init(sb + S::kPFull, 128);
-    mbar_init(sb + S::kOFull, 1);
     mbar_init(sb + S::kDrain, 1);
     *abort_flag = 0;
     fence_mbarrier_init();
   }
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tmem_alloc(sb + S::kTmemSlot, kTmemCols);
     tmem_relinquish();
   }
@@ -155,111 +190,166 @@ __global__ void __launch_bounds__(kThreads, 2)
   constexpr int kBoxes = D / 64;
   constexpr uint32_t kBlockBytes = S::kBlockBytes;
 
-  if (warp == 4) {
+  if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
     setmaxnreg_dec<kRegsOther>();
     if (lane == 0) {
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
-      uint32_t kv_seq = 0, it = 0, q_loads = 0;
+      LaneCursor cur[kLanes];
+      for (int l = 0; l < kLanes; ++l) {
+        cur[l].k = 0;
+        cursor_load(cur[l], p.items, p.n_items, l);
+      }
+      uint32_t kv_seq = 0;
+      uint32_t q_loads[kLanes] = {0, 0};
       bool ok = true;
-      for (int w = blockIdx.x; w < p.n_items && ok; w += gridDim.x, ++it) {
-        const WorkItem item = p.items[w];
-        ok = mbar_wait(sb + S::kQEmpty, (it & 1) ^ 1, wc, 1);
-        if (!ok) break;
-        ++q_loads;
-        mbar_arrive_expect_tx(sb + S::kQFull, kBlockBytes);
-        for (int b = 0; b < kBoxes; ++b)
-          tma_load_3d(sb + S::kQ + b * kBoxBytes, &tm_q, sb + S::kQFull, b * 64, item.q_row0, item.bh);
-        for (int j = 0; j < item.kv_len && ok; ++j) {
-          const int32_t kv_row = p.kv_rows[item.kv_off + j];
+      // one key or value block into the next ring stage
+      auto load_block = [&](const CUtensorMap* m, int32_t row, int32_t bh) -> bool {
+        const uint32_t st = kv_seq % kStages;
+        if (!mbar_wait(sb + S::kKvEmpty + 8 * st, ((kv_seq / kStages) & 1) ^ 1, wc, 2)) return false;
+        const uint32_t dst = sb + S::kStage0 + st * kBlockBytes;
+        const uint32_t full = sb + S::kKvFull + 8 * st;
+        mbar_arrive_expect_tx(full, kBlockBytes);
+        for (int b = 0; b < kBoxes; ++b) tma_load_3d(dst + b * kBoxBytes, m, full, b * 64, row, bh);
+        ++kv_seq;
+        return true;
+      };
+      while (ok && (cur[0].idx >= 0 || cur[1].idx >= 0)) {
 #pragma unroll
-          for (int kv = 0; kv < 2; ++kv) {
-            const uint32_t st = kv_seq % kStages;
-            const uint32_t par = ((kv_seq / kStages) & 1) ^ 1;
-            ok = mbar_wait(sb + S::kKvEmpty + 8 * st, par, wc, 2);
-            if (!ok) break;
-            const uint32_t dst = sb + S::kStage0 + st * kBlockBytes;
-            const uint32_t full = sb + S::kKvFull + 8 * st;
-            mbar_arrive_expect_tx(full, kBlockBytes);
-            const CUtensorMap* m = kv == 0 ? &tm_k : &tm_v;
-            for (int b = 0; b < kBoxes; ++b) tma_load_3d(dst + b * kBoxBytes, m, full, b * 64, kv_row, item.bh);
-            ++kv_seq;
+        for (int l = 0; l < kLanes; ++l) {  // one turn per lane, alternating
+          LaneCursor& c = cur[l];
+          if (!ok || c.idx < 0) continue;
+          if (!c.started) {
+            ok = mbar_wait(sb + S::kQEmpty + 8 * l, (q_loads[l] & 1) ^ 1, wc, 1);
+            if (!ok) continue;
+            ++q_loads[l];
+            const uint32_t qfull = sb + S::kQFull + 8 * l;
+            mbar_arrive_expect_tx(qfull, kBlockBytes);
+            for (int b = 0; b < kBoxes; ++b)
+              tma_load_3d(sb + S::kQ0 + l * kBlockBytes + b * kBoxBytes, &tm_q, qfull, b * 64, c.q_row0, c.bh);
+            ok = load_block(&tm_k, p.kv_rows[c.kv_off], c.bh);
+            c.started = true;
+          } else {
+            ok = load_block(&tm_v, p.kv_rows[c.kv_off + c.j], c.bh);
+            if (ok && c.j + 1 < c.n) ok = load_block(&tm_k, p.kv_rows[c.kv_off + c.j + 1], c.bh);
+            if (++c.j == c.n) {
+              ++c.k;
+              cursor_load(c, p.items, p.n_items, l);
+            }
           }
         }
       }
       // Drain: every load issued has landed before the CTA may exit.  Waiting on a
       // phase that already completed returns at once.
-      if (q_loads > 0) mbar_wait_drain(sb + S::kQFull, (q_loads - 1) & 1, p.limit_ns);
+      for (int q = 0; q < kLanes; ++q)
+        if (q_loads[q] > 0) mbar_wait_drain(sb + S::kQFull + 8 * q, (q_loads[q] - 1) & 1, p.limit_ns);
       for (uint32_t s = 0; s < kStages && s < kv_seq; ++s) {
         const uint32_t last = kv_seq - 1 - ((kv_seq - 1 - s) % kStages);  // last sequence number on stage s
         mbar_wait_drain(sb + S::kKvFull + 8 * s, (last / kStages) & 1, p.limit_ns);
       }
     }
     __syncwarp();
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     setmaxnreg_dec<kRegsOther>();
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
-      uint32_t kv_seq = 0, it = 0, sp = 0;
+      LaneCursor cur[kLanes];
+      for (int l = 0; l < kLanes; ++l) {
+        cur[l].k = 0;
+        cursor_load(cur[l], p.items, p.n_items, l);
+      }
+      uint32_t kv_seq = 0;
+      uint32_t q_waits[kLanes] = {0, 0}, p_waits[kLanes] = {0, 0};
       bool ok = true;
-      for (int w = blockIdx.x; w < p.n_items && ok; w += gridDim.x, ++it) {
-        const WorkItem item = p.items[w];
-        ok = mbar_wait(sb + S::kQFull, it & 1, wc, 3);
-        if (!ok) break;
+      // S_l = Q_l K^T from the next ring stage
+      auto issue_qk = [&](int l) -> bool {
+        const uint32_t st = kv_seq % kStages;
+        if (!mbar_wait(sb + S::kKvFull + 8 * st, (kv_seq / kStages) & 1, wc, 4)) return false;
         tc_fence_after();
-        for (int j = 0; j < item.kv_len && ok; ++j) {
-          // S = Q K^T
-          uint32_t st = kv_seq % kStages;
-          ok = mbar_wait(sb + S::kKvFull + 8 * st, (kv_seq / kStages) & 1, wc, 4);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t kbase = sb + S::kStage0 + st * kBlockBytes;
+        const uint32_t qbase = sb + S::kQ0 + l * kBlockBytes;
+        const uint32_t kbase = sb + S::kStage0 + st * kBlockBytes;
 #pragma unroll
-          for (int k16 = 0; k16 < D / 16; ++k16)
-            umma_ss(tmem + kSCol, kmajor_desc(sb + S::kQ, k16), kmajor_desc(kbase, k16), idesc_qk,
-                    k16 > 0 ? 1u : 0u);
-          umma_commit(sb + S::kKvEmpty + 8 * st);
-          if (j == item.kv_len - 1) umma_commit(sb + S::kQEmpty);
-          umma_commit(sb + S::kSFull);
-          ++kv_seq;
-          // O += P V once the softmax has written P
-          ok = mbar_wait(sb + S::kPFull, sp & 1, wc, 5);
-          ++sp;
-          if (!ok) break;
-          tc_fence_after();
-          st = kv_seq % kStages;
-          ok = mbar_wait(sb + S::kKvFull + 8 * st, (kv_seq / kStages) & 1, wc, 6);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t vbase = sb + S::kStage0 + st * kBlockBytes;
+        for (int k16 = 0; k16 < D / 16; ++k16)
+          umma_ss(tmem + 256 * l, kmajor_desc(qbase, k16), kmajor_desc(kbase, k16), idesc_qk, k16 > 0 ? 1u : 0u);
+        umma_commit(sb + S::kKvEmpty + 8 * st);
+        ++kv_seq;
+        return true;
+      };
+      // O_l += P_l V from the next ring stage
+      auto issue_pv = [&](int l, bool accumulate) -> bool {
+        const uint32_t st = kv_seq % kStages;
+        if (!mbar_wait(sb + S::kKvFull + 8 * st, (kv_seq / kStages) & 1, wc, 6)) return false;
+        tc_fence_after();
+        const uint32_t vbase = sb + S::kStage0 + st * kBlockBytes;
 #pragma unroll
-          for (int k16 = 0; k16 < kBlockRows / 16; ++k16)
-            umma_ts(tmem + kOCol, tmem + kSCol + k16 * 8, vmn_desc(vbase, k16), idesc_pv,
-                    (j > 0 || k16 > 0) ? 1u : 0u);
-          umma_commit(sb + S::kKvEmpty + 8 * st);
-          ++kv_seq;
+        for (int k16 = 0; k16 < kBlockRows / 16; ++k16)
+          umma_ts(tmem + 256 * l + 128, tmem + 256 * l + k16 * 8, vmn_desc(vbase, k16), idesc_pv,
+                  (accumulate || k16 > 0) ? 1u : 0u);
+        umma_commit(sb + S::kKvEmpty + 8 * st);
+        ++kv_seq;
+        return true;
+      };
+      while (ok && (cur[0].idx >= 0 || cur[1].idx >= 0)) {
+#pragma unroll
+        for (int l = 0; l < kLanes; ++l) {  // one turn per lane, alternating
+          LaneCursor& c = cur[l];
+          if (!ok || c.idx < 0) continue;
+          if (!c.started) {
+            ok = mbar_wait(sb + S::kQFull + 8 * l, q_waits[l] & 1, wc, 3);
+            ++q_waits[l];
+            if (!ok) continue;
+            tc_fence_after();
+            ok = issue_qk(l);
+            if (!ok) continue;
+            if (c.n == 1) umma_commit(sb + S::kQEmpty + 8 * l);
+            umma_commit(sb + S::kSFull + 8 * l);
+            c.started = true;
+          } else {
+            ok = mbar_wait(sb + S::kPFull + 8 * l, p_waits[l] & 1, wc, 5);
+            ++p_waits[l];
+            if (!ok) continue;
+            tc_fence_after();
+            ok = issue_pv(l, c.j > 0);
+            if (!ok) continue;
+            if (c.j + 1 < c.n) {
+              ok = issue_qk(l);
+              if (!ok) continue;
+              if (c.j + 2 == c.n) umma_commit(sb + S::kQEmpty + 8 * l);
+              umma_commit(sb + S::kSFull + 8 * l);
+            } else {
+              umma_commit(sb + S::kOFull + 8 * l);
+            }
+            if (++c.j == c.n) {
+              ++c.k;
+              cursor_load(c, p.items, p.n_items, l);
+            }
+          }
         }
-        if (ok) umma_commit(sb + S::kOFull);
       }
       // Drain: all MMAs issued by this thread complete before TMEM is freed.
       umma_commit(sb + S::kDrain);
       mbar_wait_drain(sb + S::kDrain, 0, p.limit_ns);
     }
     __syncwarp();
-  } else if (warp < 4) {
+  } else if (warp < 8) {
     // ------------------------------------------------------------ softmax + epilogue
     setmaxnreg_inc<kRegsSoftmax>();
-    const int row = threadIdx.x;                          // 0..127 = TMEM lane
-    const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const int ln = warp >> 2;                             // this warpgroup's lane
+    const int row = threadIdx.x & 127;                    // TMEM lane = query row in the block
+    const uint32_t trow = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16) + 256 * ln;
+    const uint32_t tS = trow, tO = trow + 128;
+    const uint32_t bar_s = sb + S::kSFull + 8 * ln, bar_p = sb + S::kPFull + 8 * ln, bar_o = sb + S::kOFull + 8 * ln;
     const float sl2 = p.scale_log2;
     uint32_t sphase = 0, it = 0;
     bool ok = true;
-    for (int w = blockIdx.x; w < p.n_items && ok; w += gridDim.x, ++it) {
-      const WorkItem item = p.items[w];
+    for (int32_t k = 0; ok; ++k, ++it) {
+      const int32_t idx = (k * static_cast<int32_t>(gridDim.x) + static_cast<int32_t>(blockIdx.x)) * kLanes + ln;
+      if (idx >= p.n_items) break;
+      const WorkItem item = p.items[idx];
       float m_run = -INFINITY;
       float l_run = 0.f;
       // masked path: this row's window box in tile coordinates
@@ -275,16 +365,16 @@ __global__ void __launch_bounds__(kThreads, 2)
         ws_w = min(max(aw - ew / 2, 0), p.nW - ew); we_w = ws_w + ew;
       }
       for (int j = 0; j < item.kv_len; ++j) {
-        ok = __all_sync(0xffffffffu, mbar_wait(sb + S::kSFull, sphase & 1, wc, 7));
+        ok = __all_sync(0xffffffffu, mbar_wait(bar_s, sphase & 1, wc, 7));
         ++sphase;
         if (!ok) break;
         tc_fence_after();
         // The whole score row (128 fp32) in one round trip.
         uint32_t r[128];
-        tmem_ld32_at<0>(trow + kSCol, r);
-        tmem_ld32_at<32>(trow + kSCol + 32, r);
-        tmem_ld32_at<64>(trow + kSCol + 64, r);
-        tmem_ld32_at<96>(trow + kSCol + 96, r);
+        tmem_ld32_at<0>(tS, r);
+        tmem_ld32_at<32>(tS + 32, r);
+        tmem_ld32_at<64>(tS + 64, r);
+        tmem_ld32_at<96>(tS + 96, r);
         tmem_wait_ld();
         if (MASKED) {
           const int32_t kv_row = p.kv_rows[item.kv_off + j];
@@ -304,11 +394,11 @@ __global__ void __launch_bounds__(kThreads, 2)
         // Row max: eight independent chains of three-input maxima.
         float mx8[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          float a = max3f(SV(k), SV(k + 8), SV(k + 16));
+        for (int q = 0; q < 8; ++q) {
+          float a = max3f(SV(q), SV(q + 8), SV(q + 16));
 #pragma unroll
-          for (int t = 24; t < 120; t += 16) a = max3f(a, SV(k + t), SV(k + t + 8));
-          mx8[k] = fmaxf(a, SV(k + 120));
+          for (int t = 24; t < 120; t += 16) a = max3f(a, SV(q + t), SV(q + t + 8));
+          mx8[q] = fmaxf(a, SV(q + 120));
         }
         const float mx = max3f(max3f(mx8[0], mx8[1], mx8[2]), max3f(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
         const float m_blk = mx * sl2;
@@ -330,11 +420,11 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             uint32_t o[32];
-            tmem_ld32(trow + kOCol + c * 32, o);
+            tmem_ld32(tO + c * 32, o);
             tmem_wait_ld();
 #pragma unroll
             for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
-            tmem_st32(trow + kOCol + c * 32, o);
+            tmem_st32(tO + c * 32, o);
           }
         }
         const float nm = (m_run == -INFINITY) ? 0.f : -m_run;
@@ -342,7 +432,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         // the rest on MUFU; eight partial row sums; P packed to bf16 pairs.
         float ls[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) ls[k] = 0.f;
+        for (int q = 0; q < 8; ++q) ls[q] = 0.f;
         uint32_t pk[64];
 #pragma unroll
         for (int i = 0; i < 128; i += 2) {
@@ -355,24 +445,24 @@ __global__ void __launch_bounds__(kThreads, 2)
           pk[i >> 1] = pack_bf16x2(p0, p1);
         }
 #undef SV
-        tmem_st32_at<0>(trow + kSCol, pk);
-        tmem_st32_at<32>(trow + kSCol + 32, pk);
+        tmem_st32_at<0>(tS, pk);
+        tmem_st32_at<32>(tS + 32, pk);
         l_run += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(sb + S::kPFull);
+        mbar_arrive(bar_p);
       }
       if (!ok) break;
       // epilogue: O / l -> bf16 rows (tiled order)
-      ok = __all_sync(0xffffffffu, mbar_wait(sb + S::kOFull, it & 1, wc, 8));
+      ok = __all_sync(0xffffffffu, mbar_wait(bar_o, it & 1, wc, 8));
       if (!ok) break;
       tc_fence_after();
       uint32_t o[D];
-      tmem_ld32_at<0>(trow + kOCol, o);
-      tmem_ld32_at<32>(trow + kOCol + 32, o);
+      tmem_ld32_at<0>(tO, o);
+      tmem_ld32_at<32>(tO + 32, o);
       if constexpr (D == 128) {
-        tmem_ld32_at<64>(trow + kOCol + 64, o);
-        tmem_ld32_at<96>(trow + kOCol + 96, o);
+        tmem_ld32_at<64>(tO + 64, o);
+        tmem_ld32_at<96>(tO + 96, o);
       }
       tmem_wait_ld();
       tc_fence_before();
@@ -392,13 +482,13 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
     }
   } else {
-    setmaxnreg_dec<kRegsOther>();  // warps 6-7: no role
+    setmaxnreg_dec<kRegsOther>();  // warps 10-11: no role
   }
 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 5) tmem_dealloc(tmem, kTmemCols);
+  if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
 }
 
 // Self-test kernel for the bounded wait: waits on a barrier nobody arrives on.
@@ -466,11 +556,10 @@ cudaError_t launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
   if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem)) != cudaSuccess) return e;
   if (per_sm < 1) return cudaErrorInvalidConfiguration;
-  // Two CTAs per SM by design (registers, shared memory and TMEM - 2 x 256 of 512
-  // columns - all allow exactly two).  CTAs share nothing, so a grid larger than
-  // what is resident only queues.
-  int grid = sms * 2;
-  if (grid > p.n_items) grid = p.n_items;
+  // One CTA per SM (two lanes of 128 query rows each; 512 TMEM columns).
+  int grid = sms;
+  const int pairs = (p.n_items + kLanes - 1) / kLanes;
+  if (grid > pairs) grid = pairs;
   if (grid < 1) return cudaSuccess;
   kern<<<grid, kThreads, smem, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();

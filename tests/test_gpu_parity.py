@@ -151,6 +151,19 @@ def test_attention_perhead_sampled():
     _sampled_parity(cfg, heads)
 
 
+@pytest.mark.parametrize("poly16", ["4", "6", "8"])
+def test_attention_fma_pipe_exp2_variants(poly16):
+    """Some exponentials on the FMA pipe (cubic minimax 2^f): same tolerance."""
+    import os
+    import subprocess
+    import sys
+    env = dict(os.environ, STA_EXP_POLY16=poly16)
+    here = os.path.dirname(os.path.abspath(__file__))
+    r = subprocess.run([sys.executable, os.path.join(here, "gpu_poly_check.py"), "small"], env=env,
+                       capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stdout + r.stderr
+
+
 # ------------------------------------------------------------------ behaviour
 
 
