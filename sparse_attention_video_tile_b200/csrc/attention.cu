@@ -51,10 +51,10 @@ namespace {
 using namespace ptx;
 
 constexpr int kLanes = 2;
-constexpr int kThreads = 384;       // warps 0-3 / 4-7 softmax of lane 0 / 1, 8 producer, 9 MMA, 10-11 idle
-constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
-constexpr int kStages = 4;          // key/value ring stages (K and V blocks in consumption order)
+constexpr int kThreads = 384;       // warps 0-3 / 4-7 softmax of lane 0 / 1, 8-9 producers, 10-11 MMA issuers
+constexpr int kProducerWarp0 = 8;   // + lane
+constexpr int kMmaWarp0 = 10;       // + lane; warp 10 also owns the TMEM allocation
+constexpr int kStages = 2;          // per-lane key/value ring stages (K_j, V_j, K_j+1, ... in order)
 constexpr int kTmemCols = 512;      // lane l: S at 256 l, O at 256 l + 128
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // Register split: launched at 168 per thread (384 threads, one CTA per SM);
@@ -86,64 +86,31 @@ template <int D>
 struct Smem {
   static constexpr int kBlockBytes = kBlockRows * D * 2;  // one 128-row block of Q, K or V
   static constexpr int kQ0 = 0;                            // lane l's Q at kQ0 + l * kBlockBytes
-  static constexpr int kStage0 = kLanes * kBlockBytes;
-  static constexpr int kBar = kStage0 + kStages * kBlockBytes;
-  // barriers (8 bytes each)
-  static constexpr int kQFull = kBar;                      // [lane]
-  static constexpr int kQEmpty = kQFull + 8 * kLanes;      // [lane]
-  static constexpr int kKvFull = kQEmpty + 8 * kLanes;     // [stage]
+  static constexpr int kStage0 = kLanes * kBlockBytes;     // lane l's stage s at kStage0 + (l * kStages + s) * kBlockBytes
+  static constexpr int kBar = kStage0 + kLanes * kStages * kBlockBytes;
+  // per-lane barriers (8 bytes each), lane l's copy at + l * kBarStride
+  static constexpr int kQFull = 0;
+  static constexpr int kQEmpty = 8;
+  static constexpr int kKvFull = 16;                       // [stage]
   static constexpr int kKvEmpty = kKvFull + 8 * kStages;   // [stage]
-  static constexpr int kSFull = kKvEmpty + 8 * kStages;    // [lane]
-  static constexpr int kPFull = kSFull + 8 * kLanes;       // [lane]
-  static constexpr int kOFull = kPFull + 8 * kLanes;       // [lane]
-  static constexpr int kDrain = kOFull + 8 * kLanes;
-  static constexpr int kTmemSlot = kDrain + 8;
+  static constexpr int kSFull = kKvEmpty + 8 * kStages;
+  static constexpr int kPLo = kSFull + 8;                  // P of keys 0-63 written
+  static constexpr int kPHi = kPLo + 8;                    // P of keys 64-127 written
+  static constexpr int kOFull = kPHi + 8;
+  static constexpr int kDrain = kOFull + 8;
+  static constexpr int kTurn = kDrain + 8;                 // this lane may run its exponentials
+  static constexpr int kBarStride = kTurn + 8;
+  static constexpr int kTmemSlot = kBar + kLanes * kBarStride;
   static constexpr int kAbort = kTmemSlot + 4;
   static constexpr int kEnd = kAbort + 4;
   static constexpr int kDynBytes = kEnd + 1024;  // + slack to align the base to 1024
   static_assert(kDynBytes <= 227 * 1024, "shared memory budget");
 };
 
-// Work-item cursor of one lane, shared logic of the producer and the MMA issuer.
-// Lane l of CTA c takes items (k * gridDim.x + c) * 2 + l for k = 0, 1, ...: at
-// any time the CTAs work on adjacent items (neighbouring query blocks).
-struct LaneCursor {
-  int32_t k;        // how many items this lane has finished
-  int32_t idx;      // current item, or -1 when the lane is done
-  int32_t n;        // key blocks of the current item
-  int32_t j;        // next P*V block
-  int32_t kv_off, bh, q_row0;
-  bool started;     // Q*K^T of block 0 issued
-};
-
-__device__ __forceinline__ void cursor_load(LaneCursor& c, const WorkItem* items, int32_t n_items, int lane) {
-  const int32_t idx = (c.k * static_cast<int32_t>(gridDim.x) + static_cast<int32_t>(blockIdx.x)) * kLanes + lane;
-  c.started = false;
-  c.j = 0;
-  if (idx < n_items) {
-    const WorkItem w = items[idx];
-    c.idx = idx;
-    c.n = w.kv_len;
-    c.kv_off = w.kv_off;
-    c.bh = w.bh;
-    c.q_row0 = w.q_row0;
-  } else {
-    c.idx = -1;
-  }
-}
-
-// Descriptor of a K-major bf16 operand stored as [rows][64] boxes of 128 bytes per
-// row (128-byte swizzle); k16 selects the 16-element slice along K.
-__device__ __forceinline__ uint64_t kmajor_desc(uint32_t base, int k16) {
-  const uint32_t addr = base + static_cast<uint32_t>((k16 >> 2) * (kBlockRows * 128) + (k16 & 3) * 32);
-  return sdesc_sw128(addr, 16, 1024);
-}
-
-// Descriptor of V as the MN-major B operand of P*V: rows are keys (K dim),
-// 64-wide boxes of d (N dim) at 16 KB apart; k16 selects 16 keys.
-__device__ __forceinline__ uint64_t vmn_desc(uint32_t base, int k16) {
-  const uint32_t addr = base + static_cast<uint32_t>(k16 * 16 * 128);
-  return sdesc_sw128(addr, kBlockRows * 128, 1024);
+// Item k of lane l of CTA c is (k * gridDim.x + c) * 2 + l: at any time the CTAs
+// work on adjacent items (neighbouring query blocks, overlapping windows).
+__device__ __forceinline__ int32_t lane_item(int32_t k, int lane) {
+  return (k * static_cast<int32_t>(gridDim.x) + static_cast<int32_t>(blockIdx.x)) * kLanes + lane;
 }
 
 template <int D, bool MASKED, int POLY16>
@@ -162,21 +129,24 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int l = 0; l < kLanes; ++l) {
-      mbar_init(sb + S::kQFull + 8 * l, 1);
-      mbar_init(sb + S::kQEmpty + 8 * l, 1);
-      mbar_init(sb + S::kSFull + 8 * l, 1);
-      mbar_init(sb + S::kPFull + 8 * l, 128);
-      mbar_init(sb + S::kOFull + 8 * l, 1);
+      const uint32_t b = sb + S::kBar + l * S::kBarStride;
+      mbar_init(b + S::kQFull, 1);
+      mbar_init(b + S::kQEmpty, 1);
+      for (int s = 0; s < kStages; ++s) {
+        mbar_init(b + S::kKvFull + 8 * s, 1);
+        mbar_init(b + S::kKvEmpty + 8 * s, 1);
+      }
+      mbar_init(b + S::kSFull, 1);
+      mbar_init(b + S::kPLo, 128);
+      mbar_init(b + S::kPHi, 128);
+      mbar_init(b + S::kOFull, 1);
+      mbar_init(b + S::kDrain, 1);
+      mbar_init(b + S::kTurn, 128);
     }
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(sb + S::kKvFull + 8 * s, 1);
-      mbar_init(sb + S::kKvEmpty + 8 * s, 1);
-    }
-    mbar_init(sb + S::kDrain, 1);
     *abort_flag = 0;
     fence_mbarrier_init();
   }
-  if (warp == kMmaWarp) {
+  if (warp == kMmaWarp0) {
     tmem_alloc(sb + S::kTmemSlot, kTmemCols);
     tmem_relinquish();
   }
@@ -190,149 +160,134 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int kBoxes = D / 64;
   constexpr uint32_t kBlockBytes = S::kBlockBytes;
 
-  if (warp == kProducerWarp) {
-    // ------------------------------------------------------------ producer
+  if (warp == kProducerWarp0 || warp == kProducerWarp0 + 1) {
+    // ------------------------------------------------------------ producer of one lane
     setmaxnreg_dec<kRegsOther>();
+    const int ln = warp - kProducerWarp0;
     if (lane == 0) {
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
-      LaneCursor cur[kLanes];
-      for (int l = 0; l < kLanes; ++l) {
-        cur[l].k = 0;
-        cursor_load(cur[l], p.items, p.n_items, l);
-      }
-      uint32_t kv_seq = 0;
-      uint32_t q_loads[kLanes] = {0, 0};
+      const uint32_t bars = sb + S::kBar + ln * S::kBarStride;
+      const uint32_t qdst = sb + S::kQ0 + ln * kBlockBytes;
+      const uint32_t ring = sb + S::kStage0 + ln * kStages * kBlockBytes;
+      uint32_t kv_seq = 0, q_loads = 0;
       bool ok = true;
-      // one key or value block into the next ring stage
+      // one key or value block into the lane's next ring stage
       auto load_block = [&](const CUtensorMap* m, int32_t row, int32_t bh) -> bool {
         const uint32_t st = kv_seq % kStages;
-        if (!mbar_wait(sb + S::kKvEmpty + 8 * st, ((kv_seq / kStages) & 1) ^ 1, wc, 2)) return false;
-        const uint32_t dst = sb + S::kStage0 + st * kBlockBytes;
-        const uint32_t full = sb + S::kKvFull + 8 * st;
+        if (!mbar_wait(bars + S::kKvEmpty + 8 * st, ((kv_seq / kStages) & 1) ^ 1, wc, 2)) return false;
+        const uint32_t dst = ring + st * kBlockBytes;
+        const uint32_t full = bars + S::kKvFull + 8 * st;
         mbar_arrive_expect_tx(full, kBlockBytes);
         for (int b = 0; b < kBoxes; ++b) tma_load_3d(dst + b * kBoxBytes, m, full, b * 64, row, bh);
         ++kv_seq;
         return true;
       };
-      while (ok && (cur[0].idx >= 0 || cur[1].idx >= 0)) {
-#pragma unroll
-        for (int l = 0; l < kLanes; ++l) {  // one turn per lane, alternating
-          LaneCursor& c = cur[l];
-          if (!ok || c.idx < 0) continue;
-          if (!c.started) {
-            ok = mbar_wait(sb + S::kQEmpty + 8 * l, (q_loads[l] & 1) ^ 1, wc, 1);
-            if (!ok) continue;
-            ++q_loads[l];
-            const uint32_t qfull = sb + S::kQFull + 8 * l;
-            mbar_arrive_expect_tx(qfull, kBlockBytes);
-            for (int b = 0; b < kBoxes; ++b)
-              tma_load_3d(sb + S::kQ0 + l * kBlockBytes + b * kBoxBytes, &tm_q, qfull, b * 64, c.q_row0, c.bh);
-            ok = load_block(&tm_k, p.kv_rows[c.kv_off], c.bh);
-            c.started = true;
-          } else {
-            ok = load_block(&tm_v, p.kv_rows[c.kv_off + c.j], c.bh);
-            if (ok && c.j + 1 < c.n) ok = load_block(&tm_k, p.kv_rows[c.kv_off + c.j + 1], c.bh);
-            if (++c.j == c.n) {
-              ++c.k;
-              cursor_load(c, p.items, p.n_items, l);
-            }
-          }
+      for (int32_t k = 0; ok; ++k) {
+        const int32_t idx = lane_item(k, ln);
+        if (idx >= p.n_items) break;
+        const WorkItem item = p.items[idx];
+        ok = mbar_wait(bars + S::kQEmpty, (q_loads & 1) ^ 1, wc, 1);
+        if (!ok) break;
+        ++q_loads;
+        mbar_arrive_expect_tx(bars + S::kQFull, kBlockBytes);
+        for (int b = 0; b < kBoxes; ++b)
+          tma_load_3d(qdst + b * kBoxBytes, &tm_q, bars + S::kQFull, b * 64, item.q_row0, item.bh);
+        for (int32_t j = 0; j < item.kv_len && ok; ++j) {
+          const int32_t row = p.kv_rows[item.kv_off + j];
+          ok = load_block(&tm_k, row, item.bh) && load_block(&tm_v, row, item.bh);
         }
       }
       // Drain: every load issued has landed before the CTA may exit.  Waiting on a
       // phase that already completed returns at once.
-      for (int q = 0; q < kLanes; ++q)
-        if (q_loads[q] > 0) mbar_wait_drain(sb + S::kQFull + 8 * q, (q_loads[q] - 1) & 1, p.limit_ns);
+      if (q_loads > 0) mbar_wait_drain(bars + S::kQFull, (q_loads - 1) & 1, p.limit_ns);
       for (uint32_t s = 0; s < kStages && s < kv_seq; ++s) {
         const uint32_t last = kv_seq - 1 - ((kv_seq - 1 - s) % kStages);  // last sequence number on stage s
-        mbar_wait_drain(sb + S::kKvFull + 8 * s, (last / kStages) & 1, p.limit_ns);
+        mbar_wait_drain(bars + S::kKvFull + 8 * s, (last / kStages) & 1, p.limit_ns);
       }
     }
     __syncwarp();
-  } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == kMmaWarp0 || warp == kMmaWarp0 + 1) {
+    // ------------------------------------------------------------ MMA issuer of one lane
     setmaxnreg_dec<kRegsOther>();
+    const int ln = warp - kMmaWarp0;
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
-      LaneCursor cur[kLanes];
-      for (int l = 0; l < kLanes; ++l) {
-        cur[l].k = 0;
-        cursor_load(cur[l], p.items, p.n_items, l);
-      }
-      uint32_t kv_seq = 0;
-      uint32_t q_waits[kLanes] = {0, 0}, p_waits[kLanes] = {0, 0};
-      bool ok = true;
-      // S_l = Q_l K^T from the next ring stage
-      auto issue_qk = [&](int l) -> bool {
-        const uint32_t st = kv_seq % kStages;
-        if (!mbar_wait(sb + S::kKvFull + 8 * st, (kv_seq / kStages) & 1, wc, 4)) return false;
-        tc_fence_after();
-        const uint32_t qbase = sb + S::kQ0 + l * kBlockBytes;
-        const uint32_t kbase = sb + S::kStage0 + st * kBlockBytes;
+      const uint32_t bars = sb + S::kBar + ln * S::kBarStride;
+      const uint32_t tS = tmem + 256 * ln, tO = tS + 128;
+      // Shared-memory descriptors differ only in the start-address field (bits 0-13,
+      // address >> 4; every address here is below 256 KB, so adding an offset never
+      // carries out of the field): one base descriptor per role plus offsets.
+      const uint64_t dq = sdesc_sw128(sb + S::kQ0 + ln * kBlockBytes, 16, 1024);        // K-major (Q)
+      const uint32_t ring = sb + S::kStage0 + ln * kStages * kBlockBytes;
+      const uint64_t dk0 = sdesc_sw128(ring, 16, 1024);                                   // K-major (K)
+      const uint64_t dv0 = sdesc_sw128(ring, kBlockRows * 128, 1024);                     // MN-major (V)
+      constexpr uint32_t kStageStep = kBlockBytes >> 4;
+      // slice k16 of a K-major block: 64-column boxes of 16 KB, 32 bytes per 16 columns
+      auto koff = [](int k16) -> uint64_t { return static_cast<uint64_t>(((k16 >> 2) * 16384 + (k16 & 3) * 32) >> 4); };
+      auto wait_stage = [&](uint32_t seq, int site) -> bool {
+        return mbar_wait(bars + S::kKvFull + 8 * (seq % kStages), (seq / kStages) & 1, wc, site);
+      };
+      // S = Q K^T from ring stage st
+      auto issue_qk = [&](uint32_t st) {
+        const uint64_t dk = dk0 + st * kStageStep;
 #pragma unroll
         for (int k16 = 0; k16 < D / 16; ++k16)
-          umma_ss(tmem + 256 * l, kmajor_desc(qbase, k16), kmajor_desc(kbase, k16), idesc_qk, k16 > 0 ? 1u : 0u);
-        umma_commit(sb + S::kKvEmpty + 8 * st);
-        ++kv_seq;
-        return true;
+          umma_ss(tS, dq + koff(k16), dk + koff(k16), idesc_qk, k16 > 0 ? 1u : 0u);
+        umma_commit(bars + S::kKvEmpty + 8 * st);
       };
-      // O_l += P_l V from the next ring stage
-      auto issue_pv = [&](int l, bool accumulate) -> bool {
-        const uint32_t st = kv_seq % kStages;
-        if (!mbar_wait(sb + S::kKvFull + 8 * st, (kv_seq / kStages) & 1, wc, 6)) return false;
-        tc_fence_after();
-        const uint32_t vbase = sb + S::kStage0 + st * kBlockBytes;
+      // O += P V for keys [64 h, 64 h + 64) of ring stage st (16 keys = 2 KB per slice)
+      auto issue_pv_half = [&](uint32_t st, int h, bool accumulate) {
+        const uint64_t dv = dv0 + st * kStageStep;
 #pragma unroll
-        for (int k16 = 0; k16 < kBlockRows / 16; ++k16)
-          umma_ts(tmem + 256 * l + 128, tmem + 256 * l + k16 * 8, vmn_desc(vbase, k16), idesc_pv,
+        for (int k16 = 4 * h; k16 < 4 * h + 4; ++k16)
+          umma_ts(tO, tS + k16 * 8, dv + static_cast<uint64_t>(k16 * (2048 >> 4)), idesc_pv,
                   (accumulate || k16 > 0) ? 1u : 0u);
-        umma_commit(sb + S::kKvEmpty + 8 * st);
-        ++kv_seq;
-        return true;
       };
-      while (ok && (cur[0].idx >= 0 || cur[1].idx >= 0)) {
-#pragma unroll
-        for (int l = 0; l < kLanes; ++l) {  // one turn per lane, alternating
-          LaneCursor& c = cur[l];
-          if (!ok || c.idx < 0) continue;
-          if (!c.started) {
-            ok = mbar_wait(sb + S::kQFull + 8 * l, q_waits[l] & 1, wc, 3);
-            ++q_waits[l];
-            if (!ok) continue;
-            tc_fence_after();
-            ok = issue_qk(l);
-            if (!ok) continue;
-            if (c.n == 1) umma_commit(sb + S::kQEmpty + 8 * l);
-            umma_commit(sb + S::kSFull + 8 * l);
-            c.started = true;
-          } else {
-            ok = mbar_wait(sb + S::kPFull + 8 * l, p_waits[l] & 1, wc, 5);
-            ++p_waits[l];
-            if (!ok) continue;
-            tc_fence_after();
-            ok = issue_pv(l, c.j > 0);
-            if (!ok) continue;
-            if (c.j + 1 < c.n) {
-              ok = issue_qk(l);
-              if (!ok) continue;
-              if (c.j + 2 == c.n) umma_commit(sb + S::kQEmpty + 8 * l);
-              umma_commit(sb + S::kSFull + 8 * l);
-            } else {
-              umma_commit(sb + S::kOFull + 8 * l);
-            }
-            if (++c.j == c.n) {
-              ++c.k;
-              cursor_load(c, p.items, p.n_items, l);
-            }
+      uint32_t kv_seq = 0, p_waits = 0;
+      bool ok = true;
+      for (int32_t k = 0; ok; ++k) {
+        const int32_t idx = lane_item(k, ln);
+        if (idx >= p.n_items) break;
+        const int32_t n = p.items[idx].kv_len;
+        ok = mbar_wait(bars + S::kQFull, k & 1, wc, 3) && wait_stage(kv_seq, 4);
+        if (!ok) break;
+        tc_fence_after();
+        issue_qk(kv_seq % kStages);  // S_0
+        ++kv_seq;
+        if (n == 1) umma_commit(bars + S::kQEmpty);
+        umma_commit(bars + S::kSFull);
+        for (int32_t j = 0; j < n && ok; ++j) {
+          // V_j and K_j+1 were loaded ahead: wait for them first, so that only the
+          // softmax hand-off (P_j) stands between S_j and these MMAs.
+          const bool has_k = j + 1 < n;
+          ok = wait_stage(kv_seq, 6) && (!has_k || wait_stage(kv_seq + 1, 4)) &&
+               mbar_wait(bars + S::kPLo, p_waits & 1, wc, 5);
+          if (!ok) break;
+          tc_fence_after();
+          // O += P_j V_j, the first 64 keys as soon as their P is written
+          issue_pv_half(kv_seq % kStages, 0, j > 0);
+          ok = mbar_wait(bars + S::kPHi, p_waits & 1, wc, 10);
+          ++p_waits;
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv_half(kv_seq % kStages, 1, true);
+          umma_commit(bars + S::kKvEmpty + 8 * (kv_seq % kStages));
+          ++kv_seq;
+          if (has_k) {
+            issue_qk(kv_seq % kStages);  // S_j+1 (overwrites P_j after P_j V_j, in issue order)
+            ++kv_seq;
+            if (j + 2 == n) umma_commit(bars + S::kQEmpty);
+            umma_commit(bars + S::kSFull);
           }
         }
+        if (ok) umma_commit(bars + S::kOFull);
       }
       // Drain: all MMAs issued by this thread complete before TMEM is freed.
-      umma_commit(sb + S::kDrain);
-      mbar_wait_drain(sb + S::kDrain, 0, p.limit_ns);
+      umma_commit(bars + S::kDrain);
+      mbar_wait_drain(bars + S::kDrain, 0, p.limit_ns);
     }
     __syncwarp();
   } else if (warp < 8) {
@@ -342,12 +297,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = threadIdx.x & 127;                    // TMEM lane = query row in the block
     const uint32_t trow = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16) + 256 * ln;
     const uint32_t tS = trow, tO = trow + 128;
-    const uint32_t bar_s = sb + S::kSFull + 8 * ln, bar_p = sb + S::kPFull + 8 * ln, bar_o = sb + S::kOFull + 8 * ln;
+    const uint32_t bars = sb + S::kBar + ln * S::kBarStride;
+    const uint32_t bar_s = bars + S::kSFull, bar_plo = bars + S::kPLo, bar_phi = bars + S::kPHi,
+                   bar_o = bars + S::kOFull;
     const float sl2 = p.scale_log2;
     uint32_t sphase = 0, it = 0;
     bool ok = true;
+    // Turn token: the two lanes' exponential loops alternate (lane 0 block b after
+    // lane 1 block b-1, lane 1 block b after lane 0 block b) while both have blocks,
+    // so that each has the SM's MUFU units to itself and the other lane's MMAs run
+    // meanwhile.  A lane never gets more than one phase ahead, so parity waits are
+    // exact.
+    int32_t other_total = 0;
+    for (int32_t kk = 0;; ++kk) {
+      const int32_t oi = lane_item(kk, ln ^ 1);
+      if (oi >= p.n_items) break;
+      other_total += p.items[oi].kv_len;
+    }
+    const uint32_t my_turn = bars + S::kTurn;
+    const uint32_t their_turn = sb + S::kBar + (ln ^ 1) * S::kBarStride + S::kTurn;
     for (int32_t k = 0; ok; ++k, ++it) {
-      const int32_t idx = (k * static_cast<int32_t>(gridDim.x) + static_cast<int32_t>(blockIdx.x)) * kLanes + ln;
+      const int32_t idx = lane_item(k, ln);
       if (idx >= p.n_items) break;
       const WorkItem item = p.items[idx];
       float m_run = -INFINITY;
@@ -366,6 +336,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       for (int j = 0; j < item.kv_len; ++j) {
         ok = __all_sync(0xffffffffu, mbar_wait(bar_s, sphase & 1, wc, 7));
+        const int32_t blk = static_cast<int32_t>(sphase);  // blocks of this lane before this one
         ++sphase;
         if (!ok) break;
         tc_fence_after();
@@ -428,29 +399,48 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         const float nm = (m_run == -INFINITY) ? 0.f : -m_run;
+        {
+          const int32_t need = ln == 0 ? blk - 1 : blk;  // the other lane's block to wait for
+          if (need >= 0 && need < other_total) {
+            ok = __all_sync(0xffffffffu, mbar_wait(my_turn, static_cast<uint32_t>(need & 1), wc, 9));
+            if (!ok) break;
+          }
+        }
         // p = 2^(s * scale * log2e - m): POLY16 of every 16 columns on the FMA pipe,
-        // the rest on MUFU; eight partial row sums; P packed to bf16 pairs.
+        // the rest on MUFU; eight partial row sums; P packed to bf16 pairs.  Each half
+        // of the row (64 keys) is stored and handed to the MMA issuer on its own, so
+        // P V of the first half overlaps the exponentials of the second.
         float ls[8];
 #pragma unroll
         for (int q = 0; q < 8; ++q) ls[q] = 0.f;
         uint32_t pk[64];
 #pragma unroll
-        for (int i = 0; i < 128; i += 2) {
-          const float x0 = fmaf(SV(i), sl2, nm);
-          const float x1 = fmaf(SV(i + 1), sl2, nm);
-          const float p0 = (!MASKED && (i & 15) >= 16 - POLY16) ? exp2_poly3(x0) : ex2_approx(x0);
-          const float p1 = (!MASKED && ((i + 1) & 15) >= 16 - POLY16) ? exp2_poly3(x1) : ex2_approx(x1);
-          ls[i & 7] += p0;
-          ls[(i + 1) & 7] += p1;
-          pk[i >> 1] = pack_bf16x2(p0, p1);
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+          for (int i = 64 * h; i < 64 * h + 64; i += 2) {
+            const float x0 = fmaf(SV(i), sl2, nm);
+            const float x1 = fmaf(SV(i + 1), sl2, nm);
+            const float p0 = (!MASKED && (i & 15) >= 16 - POLY16) ? exp2_poly3(x0) : ex2_approx(x0);
+            const float p1 = (!MASKED && ((i + 1) & 15) >= 16 - POLY16) ? exp2_poly3(x1) : ex2_approx(x1);
+            ls[i & 7] += p0;
+            ls[(i + 1) & 7] += p1;
+            pk[i >> 1] = pack_bf16x2(p0, p1);
+          }
+          if (h == 0) {
+            tmem_st32_at<0>(tS, pk);
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar_plo);
+          } else {
+            mbar_arrive(their_turn);  // the other lane may start its exponentials
+            tmem_st32_at<32>(tS + 32, pk);
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar_phi);
+          }
         }
 #undef SV
-        tmem_st32_at<0>(tS, pk);
-        tmem_st32_at<32>(tS + 32, pk);
         l_run += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(bar_p);
       }
       if (!ok) break;
       // epilogue: O / l -> bf16 rows (tiled order)
@@ -481,14 +471,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-  } else {
-    setmaxnreg_dec<kRegsOther>();  // warps 10-11: no role
   }
 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
+  if (warp == kMmaWarp0) tmem_dealloc(tmem, kTmemCols);
 }
 
 // Self-test kernel for the bounded wait: waits on a barrier nobody arrives on.
