@@ -32,6 +32,21 @@ if ROOT not in sys.path:
 METRIC = "STA fwd ms & TFLOPS (attended) at 30×48×80, 24 heads, d=128; % of BF16 peak"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
+# DRAM bytes (read + write) per launch of the attention kernel on the default workload, from
+# the ncu capture summarised in profiles/sta_fwd_kernel_hunyuan_4heads.md (4-head case, scaled
+# by 6 to 24 heads: traffic is per head).  Valid only for the kernel source it was taken on.
+PROFILED_TRAFFIC = {"sha1": "66ef263d91fd79626ff6e3e8e8c9b270f96e2708", "bytes_per_launch": 6 * (357.49248e6 + 104.103168e6),
+                    "workload": "hunyuan"}
+
+
+def kernel_source_sha1():
+    import hashlib
+    h = hashlib.sha1()
+    for f in ("attention.cu", "ptx.cuh"):
+        with open(os.path.join(ROOT, "sparse_attention_video_tile_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
 
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -292,6 +307,9 @@ def run_ours(args, cfg):
     peak_b = peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"])
     hbm = peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"])
     att_tflops = flops / (att_ms * 1e-3) / 1e12
+    traffic = None
+    if cfg.name == PROFILED_TRAFFIC["workload"] and kernel_source_sha1() == PROFILED_TRAFFIC["sha1"]:
+        traffic = PROFILED_TRAFFIC["bytes_per_launch"]
     reo_gbs = 2 * tensor_bytes / (reo_ms * 1e-3) / 1e9
 
     cpu = None
@@ -306,7 +324,7 @@ def run_ours(args, cfg):
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(cfg, args),
         "roofline": {"bound": "tensor", "kernel": "sta_fwd_kernel", "achieved": att_tflops, "peak": peak_s,
-                     "unit": "TFLOP/s", "frac": att_tflops / peak_s, "traffic": None,
+                     "unit": "TFLOP/s", "frac": att_tflops / peak_s, "traffic": traffic,
                      "peak_kind": f"bf16_tflops_sustained ({peaks['_source']})",
                      "frac_of_burst_peak": att_tflops / peak_b, "frac_of_2250_datasheet": att_tflops / 2250.0},
         "kernels": {"attention_ms": att_ms, "attention_tflops": att_tflops,
