@@ -54,7 +54,8 @@ typedef enum {
   STA_ERR_ARCH = 7,      /* the current device is not compute capability 10.0 (B200) */
   STA_ERR_CUDA = 8,      /* a CUDA runtime/driver call failed (message via sta_last_cuda_error) */
   STA_ERR_TIMEOUT = 9,   /* a kernel's bounded wait expired; the kernel gave up */
-  STA_ERR_ARG = 10       /* another argument is out of range (batch, heads, scale not finite ...) */
+  STA_ERR_ARG = 10,      /* another argument is out of range (batch, heads, scale not finite ...) */
+  STA_ERR_SCRATCH = 11   /* the work schedule does not fit the fixed scratch of sta_attention_fwd_noalloc */
 } sta_status;
 
 /* Human-readable name of a status code.  Static storage; never NULL. */
@@ -114,6 +115,30 @@ sta_status sta_attention_fwd(const void* q, const void* k, const void* v, void* 
                              int32_t batch, int32_t heads, int32_t d, sta_dim3 grid,
                              sta_dim3 tile, const sta_dim3* window_per_head, float scale,
                              void* stream);
+
+/*
+ * sta_attention_fwd without any device allocation by the library.  The paper has
+ * no counterpart: this entry point exists for callers that cannot let a library
+ * call cudaMalloc - code running inside a memory pool or arena it must not
+ * bypass, processes that reserve all device memory up front, or runtimes whose
+ * allocator must account for every device allocation.
+ * Same arguments, layout, semantics and errors as sta_attention_fwd, plus
+ * STA_ERR_SCRATCH when the work schedule exceeds the fixed scratch.
+ * Scratch: one static device array of 4 MiB per GPU that loads the library,
+ * held until the process exits (enough for every workload here; the largest,
+ * 24 heads at 48x48x80 with per-head windows, needs about 3 MB).  The array
+ * keeps the last call's contents: its status word is cleared on every call and
+ * the schedule is uploaded again when the configuration changes.  Calls that
+ * overlap on the GPU (different streams) race on the array; order them.
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress); make that first call before any stream capture.
+ * Bounded-wait timeouts of this variant are recorded in the scratch status word
+ * and are not reported by sta_check_device_status.
+ */
+sta_status sta_attention_fwd_noalloc(const void* q, const void* k, const void* v, void* out,
+                                     int32_t batch, int32_t heads, int32_t d, sta_dim3 grid,
+                                     sta_dim3 tile, const sta_dim3* window_per_head, float scale,
+                                     void* stream);
 
 /*
  * Synchronises `stream` and reports whether any kernel of this library gave up

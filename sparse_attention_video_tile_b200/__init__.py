@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(_HERE, "libsta.so")
 STATUS_NAMES = {
     0: "STA_OK", 1: "STA_ERR_NULL", 2: "STA_ERR_ALIGN", 3: "STA_ERR_ALIAS", 4: "STA_ERR_SHAPE",
     5: "STA_ERR_WINDOW", 6: "STA_ERR_HEADDIM", 7: "STA_ERR_ARCH", 8: "STA_ERR_CUDA",
-    9: "STA_ERR_TIMEOUT", 10: "STA_ERR_ARG",
+    9: "STA_ERR_TIMEOUT", 10: "STA_ERR_ARG", 11: "STA_ERR_SCRATCH",
 }
 STA_OK, STA_ERR_TIMEOUT = 0, 9
 

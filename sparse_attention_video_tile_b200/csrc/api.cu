@@ -167,6 +167,7 @@ const char* sta_status_str(sta_status s) {
     case STA_ERR_CUDA: return "STA_ERR_CUDA";
     case STA_ERR_TIMEOUT: return "STA_ERR_TIMEOUT";
     case STA_ERR_ARG: return "STA_ERR_ARG";
+    case STA_ERR_SCRATCH: return "STA_ERR_SCRATCH";
   }
   return "STA_ERR_UNKNOWN";
 }
