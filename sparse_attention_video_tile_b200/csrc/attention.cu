@@ -407,23 +407,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         // p = 2^(s * scale * log2e - m): POLY16 of every 16 columns on the FMA pipe,
-        // the rest on MUFU; eight partial row sums; P packed to bf16 pairs.  Each half
+        // the rest on MUFU; partial row sums; P packed to bf16 pairs.  Each half
         // of the row (64 keys) is stored and handed to the MMA issuer on its own, so
         // P V of the first half overlaps the exponentials of the second.
-        float ls[8];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) ls[q] = 0.f;
+        // x = s * scale * log2e - m and the row sums use packed fp32 pairs (one
+        // instruction per two columns); four pair-accumulators break the add chain.
+        const uint64_t sl2x2 = f32x2(sl2, sl2), nmx2 = f32x2(nm, nm);
+        uint64_t ls2[4] = {0, 0, 0, 0};
         uint32_t pk[64];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
 #pragma unroll
           for (int i = 64 * h; i < 64 * h + 64; i += 2) {
-            const float x0 = fmaf(SV(i), sl2, nm);
-            const float x1 = fmaf(SV(i + 1), sl2, nm);
+            float x0, x1;
+            f32x2_split(fma_f32x2(f32x2(SV(i), SV(i + 1)), sl2x2, nmx2), x0, x1);
             const float p0 = (!MASKED && (i & 15) >= 16 - POLY16) ? exp2_poly3(x0) : ex2_approx(x0);
             const float p1 = (!MASKED && ((i + 1) & 15) >= 16 - POLY16) ? exp2_poly3(x1) : ex2_approx(x1);
-            ls[i & 7] += p0;
-            ls[(i + 1) & 7] += p1;
+            ls2[(i >> 1) & 3] = add_f32x2(ls2[(i >> 1) & 3], f32x2(p0, p1));
             pk[i >> 1] = pack_bf16x2(p0, p1);
           }
           if (h == 0) {
@@ -440,7 +440,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
 #undef SV
-        l_run += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
+        {
+          float a0, a1, b0, b1, c0, c1, d0, d1;
+          f32x2_split(ls2[0], a0, a1);
+          f32x2_split(ls2[1], b0, b1);
+          f32x2_split(ls2[2], c0, c1);
+          f32x2_split(ls2[3], d0, d1);
+          l_run += ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
+        }
       }
       if (!ok) break;
       // epilogue: O / l -> bf16 rows (tiled order)
