@@ -65,7 +65,7 @@ constexpr int kRegsSoftmax = 208;
 constexpr int kRegsOther = 88;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsOther == kThreads * kLaunchRegs,
               "register split must match the launch");
-constexpr int kDefaultPoly16 = 0;
+constexpr int kDefaultPoly8 = 0;
 
 struct FwdParams {
   const WorkItem* items;
@@ -113,7 +113,7 @@ __device__ __forceinline__ int32_t lane_item(int32_t k, int lane) {
   return (k * static_cast<int32_t>(gridDim.x) + static_cast<int32_t>(blockIdx.x)) * kLanes + lane;
 }
 
-template <int D, bool MASKED, int POLY16>
+template <int D, bool MASKED, int POLY8>
 __global__ void __launch_bounds__(kThreads, 1)
     sta_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -406,7 +406,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!ok) break;
           }
         }
-        // p = 2^(s * scale * log2e - m): POLY16 of every 16 columns on the FMA pipe,
+        // p = 2^(s * scale * log2e - m): POLY8 of every 8 column pairs on the FMA pipe,
         // the rest on MUFU; partial row sums; P packed to bf16 pairs.  Each half
         // of the row (64 keys) is stored and handed to the MMA issuer on its own, so
         // P V of the first half overlaps the exponentials of the second.
@@ -419,10 +419,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int h = 0; h < 2; ++h) {
 #pragma unroll
           for (int i = 64 * h; i < 64 * h + 64; i += 2) {
-            float x0, x1;
-            f32x2_split(fma_f32x2(f32x2(SV(i), SV(i + 1)), sl2x2, nmx2), x0, x1);
-            const float p0 = (!MASKED && (i & 15) >= 16 - POLY16) ? exp2_poly3(x0) : ex2_approx(x0);
-            const float p1 = (!MASKED && ((i + 1) & 15) >= 16 - POLY16) ? exp2_poly3(x1) : ex2_approx(x1);
+            const uint64_t x2 = fma_f32x2(f32x2(SV(i), SV(i + 1)), sl2x2, nmx2);
+            float p0, p1;
+            if (!MASKED && ((i >> 1) & 7) >= 8 - POLY8) {
+              // x >= -125 is kept by the clamp below; x <= 8 by the rescale threshold
+              float x0, x1;
+              f32x2_split(x2, x0, x1);
+              exp2_poly3_pair(f32x2(fmaxf(x0, -125.f), fmaxf(x1, -125.f)), p0, p1);
+            } else {
+              float x0, x1;
+              f32x2_split(x2, x0, x1);
+              p0 = ex2_approx(x0);
+              p1 = ex2_approx(x1);
+            }
             ls2[(i >> 1) & 3] = add_f32x2(ls2[(i >> 1) & 3], f32x2(p0, p1));
             pk[i >> 1] = pack_bf16x2(p0, p1);
           }
@@ -532,10 +541,10 @@ bool make_tmap(CUtensorMap* m, const void* base, int64_t bh, int64_t L, int d) {
   return r == CUDA_SUCCESS;
 }
 
-template <int D, bool MASKED, int POLY16>
+template <int D, bool MASKED, int POLY8>
 cudaError_t launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
                      cudaStream_t stream) {
-  auto kern = sta_fwd_kernel<D, MASKED, POLY16>;
+  auto kern = sta_fwd_kernel<D, MASKED, POLY8>;
   const int smem = Smem<D>::kDynBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -560,14 +569,14 @@ cudaError_t launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
   return cudaGetLastError();
 }
 
-// Share of exponentials computed on the FMA pipe, in sixteenths (the rest use
-// MUFU ex2).  STA_EXP_POLY16 in the environment overrides the default; only the
-// instantiated values are accepted.
-int exp_poly16() {
+// Share of exponentials computed on the FMA pipe, in column pairs out of every 8
+// (the rest use MUFU ex2).  STA_EXP_POLY8 in the environment overrides the
+// default; only the instantiated values are accepted.
+int exp_poly8() {
   static int v = [] {
-    const char* e = std::getenv("STA_EXP_POLY16");
-    int x = e ? std::atoi(e) : kDefaultPoly16;
-    if (x != 0 && x != 4 && x != 6 && x != 8) x = kDefaultPoly16;
+    const char* e = std::getenv("STA_EXP_POLY8");
+    int x = e ? std::atoi(e) : kDefaultPoly8;
+    if (x < 0 || x > 3) x = kDefaultPoly8;
     return x;
   }();
   return v;
@@ -577,11 +586,10 @@ template <int D, bool MASKED>
 cudaError_t launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
                      cudaStream_t stream) {
   if (MASKED) return launch_t<D, MASKED, 0>(tq, tk, tv, p, stream);
-  switch (exp_poly16()) {
-    case 0: return launch_t<D, MASKED, 0>(tq, tk, tv, p, stream);
-    case 4: return launch_t<D, MASKED, 4>(tq, tk, tv, p, stream);
-    case 8: return launch_t<D, MASKED, 8>(tq, tk, tv, p, stream);
-    case 6: return launch_t<D, MASKED, 6>(tq, tk, tv, p, stream);
+  switch (exp_poly8()) {
+    case 1: return launch_t<D, MASKED, 1>(tq, tk, tv, p, stream);
+    case 2: return launch_t<D, MASKED, 2>(tq, tk, tv, p, stream);
+    case 3: return launch_t<D, MASKED, 3>(tq, tk, tv, p, stream);
     default: return launch_t<D, MASKED, 0>(tq, tk, tv, p, stream);
   }
 }

@@ -332,6 +332,23 @@ __device__ __forceinline__ uint64_t add_f32x2(uint64_t a, uint64_t b) {
   return r;
 }
 
+// 2^x for a packed pair on the FMA pipe: the same reduction and cubic as
+// exp2_poly3, with packed fp32x2 arithmetic (one instruction per pair).  For
+// finite x in [-125, 127]; callers keep x inside that range.
+__device__ __forceinline__ void exp2_poly3_pair(uint64_t x2, float& y0, float& y1) {
+  const uint64_t t2 = add_f32x2(x2, f32x2(12582912.0f, 12582912.0f));
+  const uint64_t f2 = add_f32x2(x2, fma_f32x2(t2, f32x2(-1.0f, -1.0f), f32x2(12582912.0f, 12582912.0f)));
+  uint64_t p2 = fma_f32x2(f32x2(0.0551716685295105f, 0.0551716685295105f), f2,
+                          f32x2(0.2426111251115799f, 0.2426111251115799f));
+  p2 = fma_f32x2(p2, f2, f32x2(0.6932609677314758f, 0.6932609677314758f));
+  p2 = fma_f32x2(p2, f2, f32x2(0.9999280571937561f, 0.9999280571937561f));
+  float p0, p1, t0, t1;
+  f32x2_split(p2, p0, p1);
+  f32x2_split(t2, t0, t1);
+  y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+}
+
 // Two fp32 values -> packed bf16x2 (round to nearest even); `lo` in bits 0..15.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;

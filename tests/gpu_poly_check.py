@@ -1,5 +1,5 @@
 """Run in a subprocess by test_gpu_parity: parity of one workload with the
-exponential split chosen by STA_EXP_POLY16 (read once per process)."""
+exponential split chosen by STA_EXP_POLY8 (read once per process)."""
 import os
 import sys
 

@@ -151,13 +151,13 @@ def test_attention_perhead_sampled():
     _sampled_parity(cfg, heads)
 
 
-@pytest.mark.parametrize("poly16", ["4", "6", "8"])
-def test_attention_fma_pipe_exp2_variants(poly16):
-    """Some exponentials on the FMA pipe (cubic minimax 2^f): same tolerance."""
+@pytest.mark.parametrize("poly8", ["1", "2", "3"])
+def test_attention_fma_pipe_exp2_variants(poly8):
+    """Some exponentials on the FMA pipe (cubic minimax 2^f on packed pairs): same tolerance."""
     import os
     import subprocess
     import sys
-    env = dict(os.environ, STA_EXP_POLY16=poly16)
+    env = dict(os.environ, STA_EXP_POLY8=poly8)
     here = os.path.dirname(os.path.abspath(__file__))
     r = subprocess.run([sys.executable, os.path.join(here, "gpu_poly_check.py"), "small"], env=env,
                        capture_output=True, text=True, timeout=600)
