@@ -151,6 +151,39 @@ def test_attention_perhead_sampled():
     _sampled_parity(cfg, heads)
 
 
+def test_attention_score_jumps_exercise_rescale_paths():
+    """Planted keys whose scores jump far above the running max in a later block.
+
+    Blocks after an item's first use the running max of the earlier blocks; a jump
+    of more than 2^64 takes the slow paths (first or second half of a block), smaller
+    jumps the deferred rescale.  Two query rows of an interior tile get one planted
+    key each, inside their own tile (never the first block of the window), one in
+    the first 64 keys of a 128-key block and one in the last 64.
+    """
+    cfg = W.custom_config("jumps", 1, 1, 128, (12, 24, 40), (6, 8, 8), [(1, 3, 3)])
+    q, k, v = W.make_qkv(cfg, 11)
+    # Rows dominated by one planted key output that key's value row; scaling v keeps
+    # those outputs in the magnitude range the absolute tolerance is stated for (bf16
+    # rounding of P and of the output is relative).  A wrong rescale factor would be
+    # off by 2^8 or more.
+    v = (v.float() * 0.25).to(torch.bfloat16)
+    T, H, Wd = cfg.grid
+    m = O.tiled_of_raster(cfg.grid, cfg.tile)
+    inv = np.empty_like(m)
+    inv[m] = np.arange(m.size)
+    tile_id = (1 * 3 + 1) * 5 + 2          # tile (1, 1, 2): interior in H and W
+    base = tile_id * cfg.ntile
+    for q_local, k_local in ((200, 10), (300, 100)):
+        nq, nk = int(inv[base + q_local]), int(inv[base + k_local])
+        qa = q[0, 0, nq].double()
+        lam = 110.0 / (1.4426950408889634 * cfg.scale)   # scaled score of ~110 in log2 units
+        k[0, 0, nk] = (qa * (lam / float(qa @ qa))).to(torch.bfloat16)
+    out = _run_gpu(cfg, q, k, v).float().cpu().numpy()
+    want = O.sta_attention_head(q[0, 0].double().numpy(), k[0, 0].double().numpy(), v[0, 0].double().numpy(),
+                                cfg.grid, cfg.tile, cfg.windows[0], cfg.scale)
+    _compare(out[0, 0], want, "planted score jumps")
+
+
 @pytest.mark.parametrize("poly8", ["1", "2", "3"])
 def test_attention_fma_pipe_exp2_variants(poly8):
     """Some exponentials on the FMA pipe (cubic minimax 2^f on packed pairs): same tolerance."""
