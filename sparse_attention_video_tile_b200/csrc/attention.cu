@@ -137,11 +137,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(b + S::kKvEmpty + 8 * s, 1);
       }
       mbar_init(b + S::kSFull, 1);
-      mbar_init(b + S::kPLo, 128);
-      mbar_init(b + S::kPHi, 128);
+      mbar_init(b + S::kPLo, 4);   // one arrival per softmax warp
+      mbar_init(b + S::kPHi, 4);
       mbar_init(b + S::kOFull, 1);
       mbar_init(b + S::kDrain, 1);
-      mbar_init(b + S::kTurn, 128);
+      mbar_init(b + S::kTurn, 4);
     }
     *abort_flag = 0;
     fence_mbarrier_init();
@@ -435,17 +435,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             ls2[(i >> 1) & 3] = add_f32x2(ls2[(i >> 1) & 3], f32x2(p0, p1));
             pk[i >> 1] = pack_bf16x2(p0, p1);
           }
+          // Each warp publishes its P with one elected arrival once all its lanes'
+          // TMEM stores are complete (wait::st, fence before the warp sync).
           if (h == 0) {
             tmem_st32_at<0>(tS, pk);
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(bar_plo);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_plo);
           } else {
-            mbar_arrive(their_turn);  // the other lane may start its exponentials
+            if (lane == 0) mbar_arrive(their_turn);  // the other lane may start its exponentials
             tmem_st32_at<32>(tS + 32, pk);
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(bar_phi);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_phi);
           }
         }
 #undef SV
