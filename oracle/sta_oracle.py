@@ -56,11 +56,20 @@ def raster_coords(grid: Sequence[int]) -> np.ndarray:
     return np.stack([n // (H * W), (n // W) % H, n % W], axis=1)
 
 
-def tile_grid(grid: Sequence[int], tile: Sequence[int]) -> Dim3:
-    """Number of tiles per dimension; the grid must be a multiple of the tile
-    (review reply on input resolution: latents are (a*6, b*8, c*8))."""
+def tile_grid(grid: Sequence[int], tile: Sequence[int], pad: bool = False) -> Dim3:
+    """Number of tiles per dimension.
+
+    Without padding the grid must be a multiple of the tile (review reply on input
+    resolution: latents are (a*6, b*8, c*8)).  With padding (same reply, "padding
+    with masking") the latent is conceptually padded up to the next tile multiple,
+    so the tile grid is the ceiling; the pad tokens never take part as keys.
+    """
     g, t = np.array(_dim3(grid)), np.array(_dim3(tile))
-    if np.any(t <= 0) or np.any(g <= 0) or np.any(g % t != 0):
+    if np.any(t <= 0) or np.any(g <= 0):
+        raise ValueError(f"grid {tuple(g)} and tile {tuple(t)} must be positive")
+    if pad:
+        return _dim3(-(-g // t))
+    if np.any(g % t != 0):
         raise ValueError(f"grid {tuple(g)} is not a positive multiple of tile {tuple(t)}")
     return _dim3(g // t)
 
@@ -79,10 +88,11 @@ def window_start(a: np.ndarray, weff: np.ndarray, ntiles: np.ndarray) -> np.ndar
     return np.clip(a - weff // 2, 0, np.asarray(ntiles) - weff)
 
 
-def sta_mask(q_coords: np.ndarray, k_coords: np.ndarray, grid, tile, window) -> np.ndarray:
+def sta_mask(q_coords: np.ndarray, k_coords: np.ndarray, grid, tile, window, pad: bool = False) -> np.ndarray:
     """Boolean mask[i, j]: the tile of key token j lies in the window of the tile
-    of query token i.  Coordinates are token (t, h, w) triples."""
-    ntiles = np.array(tile_grid(grid, tile))
+    of query token i.  Coordinates are token (t, h, w) triples of real tokens;
+    with ``pad`` the tile grid is that of the latent padded to tile multiples."""
+    ntiles = np.array(tile_grid(grid, tile, pad))
     tsz = np.array(_dim3(tile))
     weff = effective_window(window, ntiles)
     qa = np.asarray(q_coords) // tsz
@@ -111,12 +121,13 @@ def masked_softmax_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, mask: 
 
 def sta_attention_head(q: np.ndarray, k: np.ndarray, v: np.ndarray, grid, tile, window,
                        scale: float, rows: Optional[Iterable[int]] = None,
-                       row_block: Optional[int] = None) -> np.ndarray:
+                       row_block: Optional[int] = None, pad: bool = False) -> np.ndarray:
     """STA forward of one (batch, head): q, k, v are [L, d] in raster order.
 
     Returns fp64 output rows for ``rows`` (all rows when None), in that order.
     Work is split into row blocks only to bound memory; each row's softmax runs
-    over all L keys.
+    over all L keys.  With ``pad`` the grid need not be a tile multiple: windows
+    live on the padded tile grid and only the L real tokens are keys.
     """
     L = q.shape[0]
     coords = raster_coords(grid)
@@ -130,7 +141,7 @@ def sta_attention_head(q: np.ndarray, k: np.ndarray, v: np.ndarray, grid, tile, 
     v64 = np.asarray(v, dtype=np.float64)
     for r0 in range(0, rows.shape[0], row_block):
         sel = rows[r0:r0 + row_block]
-        mask = sta_mask(coords[sel], coords, grid, tile, window)
+        mask = sta_mask(coords[sel], coords, grid, tile, window, pad)
         out[r0:r0 + sel.shape[0]] = masked_softmax_attention(q[sel], k64, v64, mask, scale)
     return out
 
@@ -180,10 +191,11 @@ def unorder(x: np.ndarray, grid, tile) -> np.ndarray:
     return x[..., m, :]
 
 
-def attended_pairs_head(grid, tile, window) -> int:
+def attended_pairs_head(grid, tile, window, pad: bool = False) -> int:
     """Number of (query, key) token pairs one head attends, counted by visiting
-    every query tile and every key tile and testing window membership."""
-    ntiles = [int(x) for x in tile_grid(grid, tile)]
+    every query tile and every key tile and testing window membership (with
+    ``pad``, tiles count only their real tokens)."""
+    ntiles = [int(x) for x in tile_grid(grid, tile, pad)]
     ntile_tokens = int(np.prod(_dim3(tile)))
     weff = [int(x) for x in effective_window(window, ntiles)]
     starts = []
@@ -202,12 +214,30 @@ def attended_pairs_head(grid, tile, window) -> int:
                             if (s[0] <= kt < s[0] + weff[0] and s[1] <= kh < s[1] + weff[1]
                                     and s[2] <= kw < s[2] + weff[2]):
                                 n_key_tiles += 1
-                total += ntile_tokens * ntile_tokens * n_key_tiles
+                if not pad:
+                    total += ntile_tokens * ntile_tokens * n_key_tiles
+                else:
+                    qn = _real_tokens_in_tile(grid, tile, (at, ah, aw))
+                    kn = 0
+                    for kt in range(s[0], s[0] + weff[0]):
+                        for kh in range(s[1], s[1] + weff[1]):
+                            for kw in range(s[2], s[2] + weff[2]):
+                                kn += _real_tokens_in_tile(grid, tile, (kt, kh, kw))
+                    total += qn * kn
     return int(total)
 
 
-def attended_pairs(batch: int, grid, tile, windows) -> int:
-    return int(batch) * sum(attended_pairs_head(grid, tile, w) for w in windows)
+def _real_tokens_in_tile(grid, tile, a) -> int:
+    """Real (not pad) tokens of tile ``a`` of the padded tile grid."""
+    n = 1
+    for x in range(3):
+        lo = a[x] * tile[x]
+        n *= max(0, min(grid[x], lo + tile[x]) - lo)
+    return n
+
+
+def attended_pairs(batch: int, grid, tile, windows, pad: bool = False) -> int:
+    return int(batch) * sum(attended_pairs_head(grid, tile, w, pad) for w in windows)
 
 
 def attended_flops(batch: int, d: int, grid, tile, windows) -> int:

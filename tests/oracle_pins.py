@@ -116,7 +116,7 @@ def _brute_window(a, w, n):
     return set(range(s, s + we))
 
 
-def _brute_mask(grid, tile, window):
+def _brute_mask(grid, tile, window, pad=False):
     T, H, W = grid
     tt, th, tw = tile
     toks = []
@@ -124,7 +124,7 @@ def _brute_mask(grid, tile, window):
         for h in range(H):
             for w in range(W):
                 toks.append((t, h, w))
-    n = (T // tt, H // th, W // tw)
+    n = ((T + tt - 1) // tt, (H + th - 1) // th, (W + tw - 1) // tw) if pad else (T // tt, H // th, W // tw)
     L = len(toks)
     mask = np.zeros((L, L), dtype=bool)
     for i, (t, h, w) in enumerate(toks):
@@ -276,6 +276,65 @@ def pin_sampled_rows_match_full(o):
     assert np.max(np.abs(part - full[rows])) < 1e-13
 
 
+# ----------------------------------------------------------------------------- padding
+
+
+def pin_padding_golden(o):
+    for line in _read_golden("window_padded_1d.txt"):
+        lhs, rhs = line.split(":")
+        W, t, w, a = (int(x) for x in lhs.split())
+        want = [int(x) for x in rhs.split()]
+        coords = o.raster_coords((1, 1, W))
+        mask = o.sta_mask(coords, coords, (1, 1, W), (1, 1, t), (1, 1, w), pad=True)
+        got = np.nonzero(mask[a])[0].tolist()
+        assert got == want, (W, t, w, a, got, want)
+
+
+PAD_CASES = [
+    ((5, 7, 9), (2, 4, 4), (1, 1, 1)),
+    ((5, 7, 9), (2, 4, 4), (3, 3, 3)),
+    ((3, 10, 11), (2, 4, 4), (1, 3, 2)),
+    ((4, 9, 6), (3, 2, 4), (2, 3, 1)),
+]
+
+
+def pin_padding_brute_force(o):
+    for grid, tile, window in PAD_CASES:
+        coords = o.raster_coords(grid)
+        got = o.sta_mask(coords, coords, grid, tile, window, pad=True)
+        want = _brute_mask(grid, tile, window, pad=True)
+        assert np.array_equal(got, want), (grid, tile, window)
+        assert int(got.sum()) == o.attended_pairs_head(grid, tile, window, pad=True)
+
+
+def pin_padding_equals_explicit_padded_grid(o):
+    """Pad the latent explicitly (zero tokens) to a tile multiple, attend on the
+    padded grid with the unpadded rule while masking pad keys, keep real rows."""
+    for (grid, tile, window), d in zip(PAD_CASES, (8, 16, 8, 12)):
+        L = int(np.prod(grid))
+        q, k, v = _rand_qkv(L, d, seed=L)
+        gp = tuple(-(-g // t) * t for g, t in zip(grid, tile))
+        Lp = int(np.prod(gp))
+        cp = o.raster_coords(gp)
+        real = np.all(cp < np.array(grid), axis=1)
+        qp, kp, vp = (np.zeros((Lp, d)) for _ in range(3))
+        idx = np.nonzero(real)[0]  # padded raster positions of the real tokens, in raster order
+        qp[idx], kp[idx], vp[idx] = q, k, v
+        mask = o.sta_mask(cp, cp, gp, tile, window) & real[None, :]
+        outp = o.masked_softmax_attention(qp, kp, vp, mask, 0.3)
+        got = o.sta_attention_head(q, k, v, grid, tile, window, 0.3, pad=True)
+        assert np.max(np.abs(outp[idx] - got)) < 1e-12
+
+
+def pin_padding_is_noop_on_tile_multiples(o):
+    grid, tile, window, d = (4, 8, 8), (2, 4, 4), (1, 3, 1), 8
+    q, k, v = _rand_qkv(256, d, seed=31)
+    a = o.sta_attention_head(q, k, v, grid, tile, window, 0.4)
+    b = o.sta_attention_head(q, k, v, grid, tile, window, 0.4, pad=True)
+    assert np.max(np.abs(a - b)) == 0.0
+    assert o.attended_pairs_head(grid, tile, window) == o.attended_pairs_head(grid, tile, window, pad=True)
+
+
 ALL_PINS = [
     pin_index_map_golden,
     pin_index_map_properties,
@@ -289,4 +348,8 @@ ALL_PINS = [
     pin_permutation_invariance,
     pin_rows_normalised_and_hull,
     pin_sampled_rows_match_full,
+    pin_padding_golden,
+    pin_padding_brute_force,
+    pin_padding_equals_explicit_padded_grid,
+    pin_padding_is_noop_on_tile_multiples,
 ]

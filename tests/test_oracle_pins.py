@@ -76,17 +76,26 @@ def _mut_coords_hw_swapped(grid):
     return np.stack([n // (H * W), n % H, (n // H) % W], axis=1)
 
 
-def _mut_mask_transposed(q_coords, k_coords, grid, tile, window):
-    return _orig_mask(k_coords, q_coords, grid, tile, window).T
+def _mut_mask_transposed(q_coords, k_coords, grid, tile, window, pad=False):
+    return _orig_mask(k_coords, q_coords, grid, tile, window, pad).T
 
 
-def _mut_mask_token_granular(q_coords, k_coords, grid, tile, window):
+def _mut_mask_token_granular(q_coords, k_coords, grid, tile, window, pad=False):
     # token-wise sliding window: the window counted in tokens, not tiles
-    return _orig_mask(q_coords, k_coords, grid, (1, 1, 1), window)
+    return _orig_mask(q_coords, k_coords, grid, (1, 1, 1), window, pad)
+
+
+def _mut_pad_floor(grid, tile, pad=False):
+    # padded tile grid rounded down instead of up (edge tokens lose their tile)
+    g, t = np.array([int(x) for x in grid]), np.array([int(x) for x in tile])
+    if pad:
+        return tuple(int(x) for x in np.maximum(g // t, 1))
+    return _orig_tile_grid(grid, tile, pad)
 
 
 _orig_msa = O.masked_softmax_attention
 _orig_mask = O.sta_mask
+_orig_tile_grid = O.tile_grid
 
 MUTANTS = {
     "window_not_clamped": ("window_start", _mut_no_clamp),
@@ -100,6 +109,7 @@ MUTANTS = {
     "raster_h_w_swapped": ("raster_coords", _mut_coords_hw_swapped),
     "mask_transposed": ("sta_mask", _mut_mask_transposed),
     "token_granular_window": ("sta_mask", _mut_mask_token_granular),
+    "padded_tile_grid_rounded_down": ("tile_grid", _mut_pad_floor),
 }
 
 
