@@ -117,6 +117,29 @@ sta_status sta_attention_fwd(const void* q, const void* k, const void* v, void* 
                              void* stream);
 
 /*
+ * STA forward on raster-order tensors, with the tile reorder fused into the
+ * kernel's loads and stores, and padding with masking ("Fast Video Generation with
+ * Sliding Tile Attention", review reply on input resolution): the grid need not be
+ * a multiple of the tile.  The latent is treated as padded up to the next tile
+ * multiple; windows live on that padded tile grid; pad tokens are never keys and
+ * produce no output.
+ *   q, k, v, out: device bf16 [batch, heads, T*H*W, d] in raster order (token
+ *   n = (t*H + h)*W + w), 16-byte aligned; out must not overlap q, k or v.
+ *   The tile must split into 128-row slabs of whole frames: th*tw divides 128 and
+ *   tt is a multiple of 128/(th*tw) (for example (6,8,8) or (1,8,16)); other tiles
+ *   use sta_tile_reorder + sta_attention_fwd + sta_tile_unorder.
+ * Results equal those of that three-call path (up to fp32 summation order) on
+ * tile-multiple grids.  Same arithmetic, schedule caching and status reporting as
+ * sta_attention_fwd.
+ * Errors: NULL, ALIGN, ALIAS, SHAPE (tile cannot be split as above, sizes too
+ * large), WINDOW, HEADDIM, ARG, ARCH, CUDA.
+ */
+sta_status sta_attention_fwd_raster(const void* q, const void* k, const void* v, void* out,
+                                    int32_t batch, int32_t heads, int32_t d, sta_dim3 grid,
+                                    sta_dim3 tile, const sta_dim3* window_per_head, float scale,
+                                    void* stream);
+
+/*
  * sta_attention_fwd without any device allocation by the library.  The paper has
  * no counterpart: this entry point exists for callers that cannot let a library
  * call cudaMalloc - code running inside a memory pool or arena it must not

@@ -59,6 +59,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "sta_tile_reorder": (ctypes.c_int, [P, P, I64, I32, D3, D3, P]),
         "sta_tile_unorder": (ctypes.c_int, [P, P, I64, I32, D3, D3, P]),
         "sta_attention_fwd": (ctypes.c_int, [P, P, P, P, I32, I32, I32, D3, D3, ctypes.POINTER(D3), F, P]),
+        "sta_attention_fwd_raster": (ctypes.c_int, [P, P, P, P, I32, I32, I32, D3, D3, ctypes.POINTER(D3), F, P]),
         "sta_check_device_status": (ctypes.c_int, [P]),
         "sta_selftest_bounded_wait": (ctypes.c_int, [U64, P]),
         "sta_shutdown": (None, []),
@@ -174,6 +175,32 @@ def sta_attention_fwd(q, k, v, out, grid, tile, window_per_head, scale: float, s
     _check(st, "sta_attention_fwd")
 
 
+def sta_attention_fwd_raster(q, k, v, out, grid, tile, window_per_head, scale: float, stream=None) -> None:
+    """STA forward on raster-order [B, heads, T*H*W, d] bf16 CUDA tensors (tile
+    reorder fused into the kernel; grids that are not tile multiples are padded)."""
+    if q.dim() != 4:
+        raise ValueError("q must be [batch, heads, L, d]")
+    B, Hn, L, d = (int(x) for x in q.shape)
+    for name, t in (("k", k), ("v", v), ("out", out)):
+        if tuple(t.shape) != tuple(q.shape):
+            raise ValueError(f"{name} shape {tuple(t.shape)} differs from q {tuple(q.shape)}")
+    if len(window_per_head) != Hn:
+        raise ValueError("one window per head is required")
+    if L != int(np.prod([int(x) for x in grid])):
+        raise ValueError("L must equal T*H*W")
+    st = load_library().sta_attention_fwd_raster(_tensor_ptr(q, "q"), _tensor_ptr(k, "k"), _tensor_ptr(v, "v"),
+                                                 _tensor_ptr(out, "out"), B, Hn, d, _d3(grid), _d3(tile),
+                                                 _windows(window_per_head), float(scale), _stream(stream))
+    _check(st, "sta_attention_fwd_raster")
+
+
+def raster_tile_ok(tile) -> bool:
+    """Whether sta_attention_fwd_raster accepts this tile (128-row slabs of whole frames)."""
+    tt, th, tw = (int(x) for x in tile)
+    plane = th * tw
+    return 0 < plane <= 128 and 128 % plane == 0 and tt % (128 // plane) == 0
+
+
 def sta_check_device_status(stream=None) -> int:
     """Synchronises the stream; returns STA_OK or STA_ERR_TIMEOUT (raises on CUDA errors)."""
     st = load_library().sta_check_device_status(_stream(stream))
@@ -194,21 +221,29 @@ def sta_shutdown() -> None:
 
 
 def sta_forward(q, k, v, grid, tile, window_per_head, scale: Optional[float] = None,
-                stream=None, workspace: Optional[Tuple] = None):
+                stream=None, workspace: Optional[Tuple] = None, fused: Optional[bool] = None):
     """Full STA forward on raster-order [B, heads, L, d] bf16 CUDA tensors.
 
-    Reorders q, k and v to tiled order, runs the tile-windowed attention and
-    reorders the output back, all on ``stream``.  ``workspace`` may hold four
-    preallocated tensors shaped like q (tiled q, k, v and output); otherwise
-    they are allocated with torch.  Returns the raster-order output.
+    With a tile that splits into 128-row slabs of whole frames (``raster_tile_ok``)
+    and ``fused`` not False, one call does everything (``sta_attention_fwd_raster``:
+    tile reorder in the kernel's loads and stores; grids that are not tile multiples
+    are padded).  Otherwise q, k and v are reordered to tiled order, attended and
+    the output reordered back, on ``stream``; ``workspace`` may then hold four
+    preallocated tensors shaped like q (tiled q, k, v and output).  Returns the
+    raster-order output.
     """
     import torch
     if scale is None:
         scale = 1.0 / float(q.shape[-1]) ** 0.5
+    out = torch.empty_like(q)
+    if fused is None:
+        fused = raster_tile_ok(tile)
+    if fused:
+        sta_attention_fwd_raster(q, k, v, out, grid, tile, window_per_head, scale, stream)
+        return out
     if workspace is None:
         workspace = tuple(torch.empty_like(q) for _ in range(4))
     qt, kt, vt, ot = workspace
-    out = torch.empty_like(q)
     sta_tile_reorder(q, qt, grid, tile, stream)
     sta_tile_reorder(k, kt, grid, tile, stream)
     sta_tile_reorder(v, vt, grid, tile, stream)

@@ -53,9 +53,12 @@ struct CachedSchedule {
   WorkItem* d_items = nullptr;
   int32_t* d_kv_rows = nullptr;
   int16_t* d_head_win = nullptr;
+  int32_t* d_kv_mask_id = nullptr;   // padded raster schedules only
+  uint32_t* d_kv_masks = nullptr;
 };
 
-using ScheduleKey = std::tuple<int32_t, int32_t, int32_t, int32_t, int32_t, int32_t, int32_t, int32_t,
+// (raster, batch, heads, T, H, W, tt, th, tw, windows)
+using ScheduleKey = std::tuple<int32_t, int32_t, int32_t, int32_t, int32_t, int32_t, int32_t, int32_t, int32_t,
                                std::vector<int32_t>>;
 
 struct DeviceState {
@@ -71,9 +74,13 @@ void free_schedule(CachedSchedule* s) {
   if (s->d_items) cudaFree(s->d_items);
   if (s->d_kv_rows) cudaFree(s->d_kv_rows);
   if (s->d_head_win) cudaFree(s->d_head_win);
+  if (s->d_kv_mask_id) cudaFree(s->d_kv_mask_id);
+  if (s->d_kv_masks) cudaFree(s->d_kv_masks);
   s->d_items = nullptr;
   s->d_kv_rows = nullptr;
   s->d_head_win = nullptr;
+  s->d_kv_mask_id = nullptr;
+  s->d_kv_masks = nullptr;
 }
 
 // Caller holds g_mu.
@@ -99,14 +106,14 @@ cudaError_t upload(T** dst, const std::vector<T>& v) {
 
 // Caller holds g_mu.
 sta_status get_schedule(DeviceState* st, const Geometry& g, int32_t batch, int32_t heads,
-                        const sta_dim3* windows, CachedSchedule** out) {
+                        const sta_dim3* windows, bool raster, CachedSchedule** out) {
   std::vector<int32_t> wv(static_cast<size_t>(heads) * 3);
   for (int32_t h = 0; h < heads; ++h) {
     wv[h * 3 + 0] = windows[h].t;
     wv[h * 3 + 1] = windows[h].h;
     wv[h * 3 + 2] = windows[h].w;
   }
-  ScheduleKey key{batch, heads, g.T, g.H, g.W, g.tt, g.th, g.tw, std::move(wv)};
+  ScheduleKey key{raster ? 1 : 0, batch, heads, g.T, g.H, g.W, g.tt, g.th, g.tw, std::move(wv)};
   for (auto it = st->schedules.begin(); it != st->schedules.end(); ++it) {
     if (it->first == key) {
       st->schedules.splice(st->schedules.begin(), st->schedules, it);
@@ -115,13 +122,18 @@ sta_status get_schedule(DeviceState* st, const Geometry& g, int32_t batch, int32
     }
   }
   auto cs = std::make_unique<CachedSchedule>();
-  build_schedule(g, batch, heads, windows, &cs->host);
+  if (raster)
+    build_schedule_raster(g, batch, heads, windows, &cs->host);
+  else
+    build_schedule(g, batch, heads, windows, &cs->host);
   for (const WorkItem& w : cs->host.items)
     if (w.kv_len < 1) return STA_ERR_ARG;  // cannot happen: a tile always sees itself
   cudaError_t e;
   if ((e = upload(&cs->d_items, cs->host.items)) != cudaSuccess ||
       (e = upload(&cs->d_kv_rows, cs->host.kv_rows)) != cudaSuccess ||
-      (e = upload(&cs->d_head_win, cs->host.head_win)) != cudaSuccess) {
+      (e = upload(&cs->d_head_win, cs->host.head_win)) != cudaSuccess ||
+      (!cs->host.kv_masks.empty() && ((e = upload(&cs->d_kv_mask_id, cs->host.kv_mask_id)) != cudaSuccess ||
+                                      (e = upload(&cs->d_kv_masks, cs->host.kv_masks)) != cudaSuccess))) {
     free_schedule(cs.get());
     return cuda_fail(e);
   }
@@ -248,11 +260,42 @@ sta_status sta_attention_fwd(const void* q, const void* k, const void* v, void* 
   DeviceState* st = nullptr;
   if ((s = device_state(dev, &st)) != STA_OK) return s;
   CachedSchedule* cs = nullptr;
-  if ((s = get_schedule(st, g, batch, heads, window_per_head, &cs)) != STA_OK) return s;
+  if ((s = get_schedule(st, g, batch, heads, window_per_head, false, &cs)) != STA_OK) return s;
   DeviceSchedule ds{cs->d_items, cs->d_kv_rows, cs->d_head_win, static_cast<int32_t>(cs->host.items.size()),
                     cs->host.masked};
   cudaError_t e = launch_attention(q, k, v, out, batch, heads, d, g, ds, scale, st->d_err, kWaitLimitNs,
                                    static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? STA_OK : cuda_fail(e);
+}
+
+sta_status sta_attention_fwd_raster(const void* q, const void* k, const void* v, void* out, int32_t batch,
+                                    int32_t heads, int32_t d, sta_dim3 grid, sta_dim3 tile,
+                                    const sta_dim3* window_per_head, float scale, void* stream) {
+  if (!q || !k || !v || !out || !window_per_head) return STA_ERR_NULL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return STA_ERR_ALIGN;
+  if (d != 64 && d != 128) return STA_ERR_HEADDIM;
+  Geometry g;
+  sta_status s = make_geometry_padded(grid, tile, &g);
+  if (s != STA_OK) return s;
+  if (!raster_tile_ok(g.tt, g.th, g.tw) || g.ntile % kBlockRows != 0) return STA_ERR_SHAPE;
+  if (batch < 1 || heads < 1 || static_cast<int64_t>(batch) * heads > (int64_t(1) << 24)) return STA_ERR_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return STA_ERR_ARG;
+  for (int32_t h = 0; h < heads; ++h)
+    if (window_per_head[h].t < 1 || window_per_head[h].h < 1 || window_per_head[h].w < 1) return STA_ERR_WINDOW;
+  const int64_t bytes = static_cast<int64_t>(batch) * heads * g.L * d * 2;
+  if (overlaps(out, q, bytes) || overlaps(out, k, bytes) || overlaps(out, v, bytes)) return STA_ERR_ALIAS;
+  int dev = 0;
+  if ((s = check_device(&dev)) != STA_OK) return s;
+
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState* st = nullptr;
+  if ((s = device_state(dev, &st)) != STA_OK) return s;
+  CachedSchedule* cs = nullptr;
+  if ((s = get_schedule(st, g, batch, heads, window_per_head, true, &cs)) != STA_OK) return s;
+  DeviceSchedule ds{cs->d_items, cs->d_kv_rows, cs->d_head_win, static_cast<int32_t>(cs->host.items.size()), false,
+                    cs->d_kv_mask_id, cs->d_kv_masks};
+  cudaError_t e = launch_attention_raster(q, k, v, out, batch, heads, d, g, ds, scale, st->d_err, kWaitLimitNs,
+                                          static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? STA_OK : cuda_fail(e);
 }
 

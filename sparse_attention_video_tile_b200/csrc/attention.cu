@@ -70,6 +70,8 @@ constexpr int kDefaultPoly8 = 0;
 struct FwdParams {
   const WorkItem* items;
   const int32_t* kv_rows;
+  const int32_t* kv_mask_id; // per kv_rows entry: -1 or a key-validity mask (padded latents), or null
+  const uint32_t* kv_masks;  // 4 words per mask
   const int16_t* head_win;   // [heads][4]
   __nv_bfloat16* out;        // [BH, L, d] tiled order
   int32_t n_items;
@@ -77,6 +79,8 @@ struct FwdParams {
   int32_t L;
   int32_t nT, nH, nW;
   int32_t ntile;
+  // raster-order tensors: grid, tile, frames per 128-row slab
+  int32_t T, H, W, tt, th, tw, bt;
   float scale_log2;          // scale * log2(e)
   int32_t* err;
   uint64_t limit_ns;
@@ -107,13 +111,25 @@ struct Smem {
   static_assert(kDynBytes <= 227 * 1024, "shared memory budget");
 };
 
+// TMA coordinates (x, w, h, t) of the 128-row slab that starts at tiled row
+// `row` of the (padded) latent, for raster-order tensors [BH, T, H, W, d].
+struct SlabCoord {
+  int32_t w, h, t;
+};
+__device__ __forceinline__ SlabCoord slab_coord(const FwdParams& p, int32_t row) {
+  const int32_t tile = row / p.ntile;
+  const int32_t b = (row - tile * p.ntile) / kBlockRows;
+  const int32_t at = tile / (p.nH * p.nW), ah = (tile / p.nW) % p.nH, aw = tile % p.nW;
+  return SlabCoord{aw * p.tw, ah * p.th, at * p.tt + b * p.bt};
+}
+
 // Item k of lane l of CTA c is (k * gridDim.x + c) * 2 + l: at any time the CTAs
 // work on adjacent items (neighbouring query blocks, overlapping windows).
 __device__ __forceinline__ int32_t lane_item(int32_t k, int lane) {
   return (k * static_cast<int32_t>(gridDim.x) + static_cast<int32_t>(blockIdx.x)) * kLanes + lane;
 }
 
-template <int D, bool MASKED, int POLY8>
+template <int D, bool MASKED, int POLY8, bool RASTER>
 __global__ void __launch_bounds__(kThreads, 1)
     sta_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -180,7 +196,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t dst = ring + st * kBlockBytes;
         const uint32_t full = bars + S::kKvFull + 8 * st;
         mbar_arrive_expect_tx(full, kBlockBytes);
-        for (int b = 0; b < kBoxes; ++b) tma_load_3d(dst + b * kBoxBytes, m, full, b * 64, row, bh);
+        if constexpr (RASTER) {
+          const SlabCoord c = slab_coord(p, row);
+          for (int b = 0; b < kBoxes; ++b) tma_load_5d(dst + b * kBoxBytes, m, full, b * 64, c.w, c.h, c.t, bh);
+        } else {
+          for (int b = 0; b < kBoxes; ++b) tma_load_3d(dst + b * kBoxBytes, m, full, b * 64, row, bh);
+        }
         ++kv_seq;
         return true;
       };
@@ -192,8 +213,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         ++q_loads;
         mbar_arrive_expect_tx(bars + S::kQFull, kBlockBytes);
-        for (int b = 0; b < kBoxes; ++b)
-          tma_load_3d(qdst + b * kBoxBytes, &tm_q, bars + S::kQFull, b * 64, item.q_row0, item.bh);
+        if constexpr (RASTER) {
+          const SlabCoord c = slab_coord(p, item.q_row0);
+          for (int b = 0; b < kBoxes; ++b)
+            tma_load_5d(qdst + b * kBoxBytes, &tm_q, bars + S::kQFull, b * 64, c.w, c.h, c.t, item.bh);
+        } else {
+          for (int b = 0; b < kBoxes; ++b)
+            tma_load_3d(qdst + b * kBoxBytes, &tm_q, bars + S::kQFull, b * 64, item.q_row0, item.bh);
+        }
         for (int32_t j = 0; j < item.kv_len && ok; ++j) {
           const int32_t row = p.kv_rows[item.kv_off + j];
           ok = load_block(&tm_k, row, item.bh) && load_block(&tm_v, row, item.bh);
@@ -347,6 +374,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32_at<64>(tS + 64, r);
         tmem_ld32_at<96>(tS + 96, r);
         tmem_wait_ld();
+        if (!MASKED && p.kv_mask_id != nullptr) {
+          // padded latent: keys of pad tokens in this block do not exist
+          const int32_t mid = p.kv_mask_id[item.kv_off + j];
+          if (mid >= 0) {
+            const uint4 mw = *reinterpret_cast<const uint4*>(p.kv_masks + 4 * mid);
+            const uint32_t words[4] = {mw.x, mw.y, mw.z, mw.w};
+#pragma unroll
+            for (int i = 0; i < 128; ++i)
+              if (!((words[i >> 5] >> (i & 31)) & 1u)) r[i] = __float_as_uint(-INFINITY);
+          }
+        }
         if (MASKED) {
           const int32_t kv_row = p.kv_rows[item.kv_off + j];
 #pragma unroll
@@ -478,8 +516,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       const float inv_l = 1.0f / l_run;
       const int32_t qrow = item.q_row0 + row;
-      if (qrow < p.L) {
-        uint4* dst = reinterpret_cast<uint4*>(p.out + (static_cast<int64_t>(item.bh) * p.L + qrow) * D);
+      int64_t out_row = -1;  // destination row, or -1 for no real token
+      if constexpr (RASTER) {
+        const int32_t tile = qrow / p.ntile, local = qrow - tile * p.ntile;
+        const int32_t at = tile / (p.nH * p.nW), ah = (tile / p.nW) % p.nH, aw = tile % p.nW;
+        const int32_t t = at * p.tt + local / (p.th * p.tw);
+        const int32_t hh = ah * p.th + (local / p.tw) % p.th;
+        const int32_t w = aw * p.tw + local % p.tw;
+        if (t < p.T && hh < p.H && w < p.W)
+          out_row = ((static_cast<int64_t>(item.bh) * p.T + t) * p.H + hh) * p.W + w;
+      } else if (qrow < p.L) {
+        out_row = static_cast<int64_t>(item.bh) * p.L + qrow;
+      }
+      if (out_row >= 0) {
+        uint4* dst = reinterpret_cast<uint4*>(p.out + out_row * D);
 #pragma unroll
         for (int c = 0; c < D / 8; ++c) {
           uint4 v4;
@@ -545,10 +595,29 @@ bool make_tmap(CUtensorMap* m, const void* base, int64_t bh, int64_t L, int d) {
   return r == CUDA_SUCCESS;
 }
 
-template <int D, bool MASKED, int POLY8>
+// Tensor map of a raster-order [BH, T, H, W, d] bf16 tensor whose box is one
+// 128-row slab of a tile (bt frames x th x tw tokens) x 64 columns, 128-byte
+// swizzle: the box's rows come out in tile-local raster order, the tiled order.
+// Coordinates past the grid (pad tokens of a padded latent) read as zero.
+bool make_tmap_raster(CUtensorMap* m, const void* base, int64_t bh, const Geometry& g, int d, int bt) {
+  auto fn = get_encode_fn();
+  if (!fn) return false;
+  const cuuint64_t row = static_cast<cuuint64_t>(d) * 2;
+  cuuint64_t dims[5] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(g.W), static_cast<cuuint64_t>(g.H),
+                        static_cast<cuuint64_t>(g.T), static_cast<cuuint64_t>(bh)};
+  cuuint64_t strides[4] = {row, row * g.W, row * g.W * g.H, row * g.W * g.H * g.T};
+  cuuint32_t box[5] = {64, static_cast<cuuint32_t>(g.tw), static_cast<cuuint32_t>(g.th), static_cast<cuuint32_t>(bt), 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int D, bool MASKED, int POLY8, bool RASTER>
 cudaError_t launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
                      cudaStream_t stream) {
-  auto kern = sta_fwd_kernel<D, MASKED, POLY8>;
+  auto kern = sta_fwd_kernel<D, MASKED, POLY8, RASTER>;
   const int smem = Smem<D>::kDynBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -575,27 +644,46 @@ cudaError_t launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
 
 // Share of exponentials computed on the FMA pipe, in column pairs out of every 8
 // (the rest use MUFU ex2).  STA_EXP_POLY8 in the environment overrides the
-// default; only the instantiated values are accepted.
+// default; only the instantiated values (0, 1) are accepted.
 int exp_poly8() {
   static int v = [] {
     const char* e = std::getenv("STA_EXP_POLY8");
     int x = e ? std::atoi(e) : kDefaultPoly8;
-    if (x < 0 || x > 3) x = kDefaultPoly8;
+    if (x < 0 || x > 1) x = kDefaultPoly8;
     return x;
   }();
   return v;
 }
 
-template <int D, bool MASKED>
+template <int D, bool MASKED, bool RASTER>
 cudaError_t launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
                      cudaStream_t stream) {
-  if (MASKED) return launch_t<D, MASKED, 0>(tq, tk, tv, p, stream);
-  switch (exp_poly8()) {
-    case 1: return launch_t<D, MASKED, 1>(tq, tk, tv, p, stream);
-    case 2: return launch_t<D, MASKED, 2>(tq, tk, tv, p, stream);
-    case 3: return launch_t<D, MASKED, 3>(tq, tk, tv, p, stream);
-    default: return launch_t<D, MASKED, 0>(tq, tk, tv, p, stream);
-  }
+  if (MASKED) return launch_t<D, MASKED, 0, RASTER>(tq, tk, tv, p, stream);
+  if (exp_poly8() == 1) return launch_t<D, MASKED, 1, RASTER>(tq, tk, tv, p, stream);
+  return launch_t<D, MASKED, 0, RASTER>(tq, tk, tv, p, stream);
+}
+
+FwdParams make_params(void* out, int32_t heads, const Geometry& g, const DeviceSchedule& s, float scale,
+                      int32_t* err_flag, uint64_t limit_ns) {
+  FwdParams p;
+  p.items = s.items;
+  p.kv_rows = s.kv_rows;
+  p.kv_mask_id = s.kv_mask_id;
+  p.kv_masks = s.kv_masks;
+  p.head_win = s.head_win;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.n_items = s.n_items;
+  p.heads = heads;
+  p.L = static_cast<int32_t>(g.L);
+  p.nT = g.nT; p.nH = g.nH; p.nW = g.nW;
+  p.ntile = g.ntile;
+  p.T = g.T; p.H = g.H; p.W = g.W;
+  p.tt = g.tt; p.th = g.th; p.tw = g.tw;
+  p.bt = (g.th * g.tw) > 0 ? kBlockRows / (g.th * g.tw) : 0;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.err = err_flag;
+  p.limit_ns = limit_ns;
+  return p;
 }
 
 }  // namespace
@@ -607,23 +695,25 @@ cudaError_t launch_attention(const void* q, const void* k, const void* v, void* 
   CUtensorMap tq, tk, tv;
   if (!make_tmap(&tq, q, bh, g.L, d) || !make_tmap(&tk, k, bh, g.L, d) || !make_tmap(&tv, v, bh, g.L, d))
     return cudaErrorInvalidValue;
-  FwdParams p;
-  p.items = s.items;
-  p.kv_rows = s.kv_rows;
-  p.head_win = s.head_win;
-  p.out = static_cast<__nv_bfloat16*>(out);
-  p.n_items = s.n_items;
-  p.heads = heads;
-  p.L = static_cast<int32_t>(g.L);
-  p.nT = g.nT; p.nH = g.nH; p.nW = g.nW;
-  p.ntile = g.ntile;
-  p.scale_log2 = scale * 1.4426950408889634f;
-  p.err = err_flag;
-  p.limit_ns = limit_ns;
-  if (d == 128) {
-    return s.masked ? launch_d<128, true>(tq, tk, tv, p, stream) : launch_d<128, false>(tq, tk, tv, p, stream);
-  }
-  return s.masked ? launch_d<64, true>(tq, tk, tv, p, stream) : launch_d<64, false>(tq, tk, tv, p, stream);
+  const FwdParams p = make_params(out, heads, g, s, scale, err_flag, limit_ns);
+  if (d == 128)
+    return s.masked ? launch_d<128, true, false>(tq, tk, tv, p, stream) : launch_d<128, false, false>(tq, tk, tv, p, stream);
+  return s.masked ? launch_d<64, true, false>(tq, tk, tv, p, stream) : launch_d<64, false, false>(tq, tk, tv, p, stream);
+}
+
+cudaError_t launch_attention_raster(const void* q, const void* k, const void* v, void* out, int32_t batch,
+                                    int32_t heads, int32_t d, const Geometry& g, const DeviceSchedule& s,
+                                    float scale, int32_t* err_flag, uint64_t limit_ns, cudaStream_t stream) {
+  if (s.masked || !raster_tile_ok(g.tt, g.th, g.tw) || g.ntile % kBlockRows != 0) return cudaErrorInvalidValue;
+  const int64_t bh = static_cast<int64_t>(batch) * heads;
+  const int bt = kBlockRows / (g.th * g.tw);
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap_raster(&tq, q, bh, g, d, bt) || !make_tmap_raster(&tk, k, bh, g, d, bt) ||
+      !make_tmap_raster(&tv, v, bh, g, d, bt))
+    return cudaErrorInvalidValue;
+  const FwdParams p = make_params(out, heads, g, s, scale, err_flag, limit_ns);
+  if (d == 128) return launch_d<128, false, true>(tq, tk, tv, p, stream);
+  return launch_d<64, false, true>(tq, tk, tv, p, stream);
 }
 
 cudaError_t launch_selftest_wait(int32_t* err_flag, uint64_t limit_ns, cudaStream_t stream) {

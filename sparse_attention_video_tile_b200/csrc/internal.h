@@ -14,13 +14,20 @@ namespace sta {
 struct Geometry {
   int32_t T, H, W;        // grid in tokens
   int32_t tt, th, tw;     // tile in tokens
-  int32_t nT, nH, nW;     // tile grid
+  int32_t nT, nH, nW;     // tile grid (of the padded latent when padded)
   int32_t ntile;          // tokens per tile
-  int64_t L;              // tokens
+  int64_t L;              // real tokens T * H * W
+  int64_t Lpad;           // rows of the tiled order: nT * nH * nW * ntile (= L unless padded)
+  bool padded;            // grid is not a tile multiple
 };
 
-// Validates and fills a Geometry; STA_OK or STA_ERR_SHAPE.
+// Validates and fills a Geometry; the grid must be a tile multiple.
+// STA_OK or STA_ERR_SHAPE.
 sta_status make_geometry(sta_dim3 grid, sta_dim3 tile, Geometry* g);
+
+// Same, but a grid that is not a tile multiple is padded up to the next multiple
+// ("padding with masking").
+sta_status make_geometry_padded(sta_dim3 grid, sta_dim3 tile, Geometry* g);
 
 // One unit of work of the attention kernel: a block of 128 query rows of one
 // (batch, head), with the list of 128-key blocks it attends.
@@ -37,6 +44,10 @@ struct HostSchedule {
   std::vector<WorkItem> items;         // sorted by decreasing cost (kv_len), stable
   std::vector<int32_t> kv_rows;        // first row (tiled order) of each 128-key block
   std::vector<int16_t> head_win;       // [heads][4]: effective window (t, h, w), 0
+  // Padded latents only: per entry of kv_rows, -1 if every key of the block is a real
+  // token, else the index of a 128-bit validity mask (4 words, bit i = key i is real).
+  std::vector<int32_t> kv_mask_id;
+  std::vector<uint32_t> kv_masks;
   int64_t attended_pairs = 0;
 };
 
@@ -46,6 +57,20 @@ constexpr int kBlockRows = 128;   // query rows per work item and keys per key b
 // the window (see schedule.cpp).
 void build_schedule(const Geometry& g, int32_t batch, int32_t heads, const sta_dim3* windows,
                     HostSchedule* out);
+
+// Window enumerator of the raster-order kernel: Ntile must be a multiple of 128 and
+// the grid may be padded.  Key blocks without real tokens are left out, partly
+// padded ones get a validity mask, and query blocks without real rows get no item.
+void build_schedule_raster(const Geometry& g, int32_t batch, int32_t heads, const sta_dim3* windows,
+                           HostSchedule* out);
+
+// Whether a tile splits into 128-row slabs of whole frames (th * tw divides 128 and
+// tt is a multiple of 128 / (th * tw)): the raster-order kernel loads each slab as
+// one TMA box.
+inline bool raster_tile_ok(int32_t tt, int32_t th, int32_t tw) {
+  const int32_t plane = th * tw;
+  return plane > 0 && plane <= kBlockRows && kBlockRows % plane == 0 && tt % (kBlockRows / plane) == 0;
+}
 
 // Effective window start (first tile) in one dimension.
 inline int32_t window_start_1d(int32_t a, int32_t weff, int32_t n) {
@@ -65,12 +90,22 @@ struct DeviceSchedule {
   const int16_t* head_win;
   int32_t n_items;
   bool masked;
+  const int32_t* kv_mask_id = nullptr;   // padded latents only
+  const uint32_t* kv_masks = nullptr;
 };
 
+// Attention on tiled-order tensors ([BH, L, d]).
 cudaError_t launch_attention(const void* q, const void* k, const void* v, void* out,
                              int32_t batch, int32_t heads, int32_t d, const Geometry& g,
                              const DeviceSchedule& s, float scale, int32_t* err_flag,
                              uint64_t limit_ns, cudaStream_t stream);
+
+// Attention on raster-order tensors ([BH, T, H, W, d]): the tile reorder is done by
+// the TMA loads and the epilogue's addressing; pad tokens read as zeros.
+cudaError_t launch_attention_raster(const void* q, const void* k, const void* v, void* out,
+                                    int32_t batch, int32_t heads, int32_t d, const Geometry& g,
+                                    const DeviceSchedule& s, float scale, int32_t* err_flag,
+                                    uint64_t limit_ns, cudaStream_t stream);
 
 cudaError_t launch_selftest_wait(int32_t* err_flag, uint64_t limit_ns, cudaStream_t stream);
 

@@ -19,6 +19,7 @@
 // a persistent grid balances per-head windows of different sizes, and CTAs that
 // run at the same time share key/value tiles in L2.
 #include <algorithm>
+#include <array>
 #include <map>
 #include <set>
 #include <tuple>
@@ -38,6 +39,26 @@ sta_status make_geometry(sta_dim3 grid, sta_dim3 tile, Geometry* g) {
   g->nT = grid.t / tile.t; g->nH = grid.h / tile.h; g->nW = grid.w / tile.w;
   g->ntile = tile.t * tile.h * tile.w;
   g->L = L;
+  g->Lpad = L;
+  g->padded = false;
+  return STA_OK;
+}
+
+sta_status make_geometry_padded(sta_dim3 grid, sta_dim3 tile, Geometry* g) {
+  if (grid.t <= 0 || grid.h <= 0 || grid.w <= 0 || tile.t <= 0 || tile.h <= 0 || tile.w <= 0)
+    return STA_ERR_SHAPE;
+  const int64_t nT = (grid.t + tile.t - 1) / tile.t, nH = (grid.h + tile.h - 1) / tile.h,
+                nW = (grid.w + tile.w - 1) / tile.w;
+  const int64_t ntile = static_cast<int64_t>(tile.t) * tile.h * tile.w;
+  const int64_t Lpad = nT * nH * nW * ntile;
+  if (Lpad >= (int64_t(1) << 31) - kBlockRows || ntile >= (int64_t(1) << 31)) return STA_ERR_SHAPE;
+  g->T = grid.t; g->H = grid.h; g->W = grid.w;
+  g->tt = tile.t; g->th = tile.h; g->tw = tile.w;
+  g->nT = static_cast<int32_t>(nT); g->nH = static_cast<int32_t>(nH); g->nW = static_cast<int32_t>(nW);
+  g->ntile = static_cast<int32_t>(ntile);
+  g->L = static_cast<int64_t>(grid.t) * grid.h * grid.w;
+  g->Lpad = Lpad;
+  g->padded = Lpad != g->L;
   return STA_OK;
 }
 
@@ -125,6 +146,112 @@ void build_schedule(const Geometry& g, int32_t batch, int32_t heads, const sta_d
       const auto& per_qb = lists[eff[h]];
       for (int32_t qb = 0; qb < n_qblocks; ++qb)
         s->items.push_back(WorkItem{b * heads + h, qb * kBlockRows, per_qb[qb].first, per_qb[qb].second});
+    }
+  std::stable_sort(s->items.begin(), s->items.end(),
+                   [](const WorkItem& x, const WorkItem& y) { return x.kv_len > y.kv_len; });
+}
+
+namespace {
+
+// Whether tiled row m (of the padded latent) is a real token.
+bool row_is_real(const Geometry& g, int64_t m) {
+  const int64_t tile = m / g.ntile;
+  const int32_t local = static_cast<int32_t>(m - tile * g.ntile);
+  const int32_t at = static_cast<int32_t>(tile / (static_cast<int64_t>(g.nH) * g.nW));
+  const int32_t ah = static_cast<int32_t>((tile / g.nW) % g.nH);
+  const int32_t aw = static_cast<int32_t>(tile % g.nW);
+  const int32_t lt = local / (g.th * g.tw), lh = (local / g.tw) % g.th, lw = local % g.tw;
+  return at * g.tt + lt < g.T && ah * g.th + lh < g.H && aw * g.tw + lw < g.W;
+}
+
+}  // namespace
+
+void build_schedule_raster(const Geometry& g, int32_t batch, int32_t heads, const sta_dim3* windows,
+                           HostSchedule* s) {
+  s->masked = false;
+  s->items.clear();
+  s->kv_rows.clear();
+  s->kv_mask_id.clear();
+  s->kv_masks.clear();
+  s->head_win.assign(static_cast<size_t>(heads) * 4, 0);
+  s->attended_pairs = 0;
+
+  const int32_t n_tiles = g.nT * g.nH * g.nW;
+  const int32_t bpt = g.ntile / kBlockRows;  // 128-row blocks per tile
+  // Per block of the padded tiled order: real rows and, when partial, a mask id.
+  std::vector<int32_t> real_rows(static_cast<size_t>(n_tiles) * bpt, kBlockRows);
+  std::vector<int32_t> block_mask(static_cast<size_t>(n_tiles) * bpt, -1);
+  if (g.padded) {
+    std::map<std::array<uint32_t, 4>, int32_t> dedup;
+    for (int64_t blk = 0; blk < static_cast<int64_t>(n_tiles) * bpt; ++blk) {
+      std::array<uint32_t, 4> bits{0, 0, 0, 0};
+      int32_t n = 0;
+      for (int32_t i = 0; i < kBlockRows; ++i)
+        if (row_is_real(g, blk * kBlockRows + i)) {
+          bits[i >> 5] |= 1u << (i & 31);
+          ++n;
+        }
+      real_rows[blk] = n;
+      if (n > 0 && n < kBlockRows) {
+        auto it = dedup.find(bits);
+        if (it == dedup.end()) {
+          const int32_t id = static_cast<int32_t>(s->kv_masks.size() / 4);
+          for (uint32_t w : bits) s->kv_masks.push_back(w);
+          it = dedup.emplace(bits, id).first;
+        }
+        block_mask[blk] = it->second;
+      }
+    }
+  }
+
+  std::map<Eff, std::vector<std::pair<int32_t, int32_t>>> lists;  // per query tile: (off, len)
+  std::vector<int32_t> tiles;
+  std::vector<Eff> eff(heads);
+  for (int32_t h = 0; h < heads; ++h) {
+    Eff e{std::min(windows[h].t, g.nT), std::min(windows[h].h, g.nH), std::min(windows[h].w, g.nW)};
+    eff[h] = e;
+    s->head_win[h * 4 + 0] = static_cast<int16_t>(e.t);
+    s->head_win[h * 4 + 1] = static_cast<int16_t>(e.h);
+    s->head_win[h * 4 + 2] = static_cast<int16_t>(e.w);
+    if (lists.count(e)) continue;
+    std::vector<std::pair<int32_t, int32_t>>& per_tile = lists[e];
+    per_tile.resize(n_tiles);
+    for (int32_t qt = 0; qt < n_tiles; ++qt) {
+      window_tiles(g, e, qt, &tiles);
+      const int32_t off = static_cast<int32_t>(s->kv_rows.size());
+      for (int32_t kt : tiles)
+        for (int32_t b = 0; b < bpt; ++b) {
+          const int64_t blk = static_cast<int64_t>(kt) * bpt + b;
+          if (real_rows[blk] == 0) continue;  // nothing but pad keys
+          s->kv_rows.push_back(static_cast<int32_t>(blk * kBlockRows));
+          s->kv_mask_id.push_back(block_mask[blk]);
+        }
+      per_tile[qt] = {off, static_cast<int32_t>(s->kv_rows.size()) - off};
+    }
+  }
+  // Attended pairs: real query rows times real keys of their window.
+  for (int32_t h = 0; h < heads; ++h) {
+    const auto& per_tile = lists[eff[h]];
+    for (int32_t qt = 0; qt < n_tiles; ++qt) {
+      int64_t keys = 0;
+      for (int32_t i = per_tile[qt].first; i < per_tile[qt].first + per_tile[qt].second; ++i)
+        keys += real_rows[s->kv_rows[i] / kBlockRows];
+      int64_t qrows = 0;
+      for (int32_t b = 0; b < bpt; ++b) qrows += real_rows[static_cast<int64_t>(qt) * bpt + b];
+      s->attended_pairs += static_cast<int64_t>(batch) * qrows * keys;
+    }
+  }
+
+  s->items.reserve(static_cast<size_t>(batch) * heads * n_tiles * bpt);
+  for (int32_t b = 0; b < batch; ++b)
+    for (int32_t h = 0; h < heads; ++h) {
+      const auto& per_tile = lists[eff[h]];
+      for (int32_t qt = 0; qt < n_tiles; ++qt)
+        for (int32_t qb = 0; qb < bpt; ++qb) {
+          if (real_rows[static_cast<int64_t>(qt) * bpt + qb] == 0) continue;  // only pad rows
+          s->items.push_back(WorkItem{b * heads + h, (qt * bpt + qb) * kBlockRows, per_tile[qt].first,
+                                      per_tile[qt].second});
+        }
     }
   std::stable_sort(s->items.begin(), s->items.end(),
                    [](const WorkItem& x, const WorkItem& y) { return x.kv_len > y.kv_len; });
