@@ -1,8 +1,10 @@
 """Benchmark of the Sliding Tile Attention forward path on B200.
 
-One step = the whole hot path on one batch of synthetic input: reorder q, k
-and v to tiled order, tile-windowed attention, reorder the output back.  The
-default workload is the HunyuanVideo-shaped one (latent 30x48x80 = 115200
+One step = the whole hot path on one batch of synthetic input: tile reorder of
+q, k and v, tile-windowed attention, reorder of the output back.  With tiles that
+split into 128-row slabs of whole frames (the default workload) that is one
+launch of the fused raster-order kernel; --three-call times the separate
+reorder / tiled attention / unorder kernels instead.  The default workload is the HunyuanVideo-shaped one (latent 30x48x80 = 115200
 tokens, tile (6,8,8), window (3,3,3) tiles, 24 heads, d = 128, bf16).
 
 value = attended FLOPs (4 * d * attended query-key pairs) of all ranks per
@@ -32,10 +34,11 @@ if ROOT not in sys.path:
 METRIC = "STA fwd ms & TFLOPS (attended) at 30×48×80, 24 heads, d=128; % of BF16 peak"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-# DRAM bytes (read + write) per launch of the attention kernel on the default workload, from
-# the ncu capture summarised in profiles/sta_fwd_kernel_hunyuan_4heads.md (4-head case, scaled
-# by 6 to 24 heads: traffic is per head).  Valid only for the kernel source it was taken on.
-PROFILED_TRAFFIC = {"sha1": "66ef263d91fd79626ff6e3e8e8c9b270f96e2708", "bytes_per_launch": 6 * (357.49248e6 + 104.103168e6),
+# DRAM bytes (read + write) per launch of the fused raster-order attention kernel on the default
+# workload, from the ncu capture summarised in profiles/sta_fwd_kernel_hunyuan_4heads.md (4-head
+# case, scaled by 6 to 24 heads: traffic is per head).  Valid only for the kernel source it was
+# taken on.
+PROFILED_TRAFFIC = {"sha1": "6a4584f45c0e95d62aebbcf8b8c0db458af052fb", "bytes_per_launch": 6 * (360.189696e6 + 101.390592e6),
                     "workload": "hunyuan"}
 
 
@@ -224,11 +227,16 @@ def run_ours(args, cfg):
     flops = 4.0 * cfg.d * sta.sta_attended_pairs(cfg.batch, cfg.heads, grid, tile, wins)
     tensor_bytes = q.numel() * q.element_size()
 
+    # One step = the whole hot path on one batch: with a tile that splits into 128-row
+    # slabs of whole frames, one launch of the fused raster-order kernel (tile reorder
+    # in its TMA loads and output addressing); otherwise reorder q, k, v, tiled
+    # attention, unorder (five launches).
+    fused = sta.raster_tile_ok(tile) and not args.three_call
     ev = {n: [] for n in ("r0", "r1", "a0", "a1", "u0", "u1")}
 
-    def step(record: bool):
+    def step_three(record: bool, store=ev):
         if record:
-            e = {n: torch.cuda.Event(enable_timing=True) for n in ev}
+            e = {n: torch.cuda.Event(enable_timing=True) for n in store}
             e["r0"].record(stream)
         sta.sta_tile_reorder(q, qt, grid, tile, stream)
         sta.sta_tile_reorder(k, kt, grid, tile, stream)
@@ -243,8 +251,20 @@ def run_ours(args, cfg):
         sta.sta_tile_unorder(ot, out, grid, tile, stream)
         if record:
             e["u1"].record(stream)
-            for n in ev:
-                ev[n].append(e[n])
+            for n in store:
+                store[n].append(e[n])
+
+    def step_fused(record: bool):
+        if record:
+            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+        sta.sta_attention_fwd_raster(q, k, v, out, grid, tile, wins, scale, stream)
+        if record:
+            a1.record(stream)
+            ev["a0"].append(a0)
+            ev["a1"].append(a1)
+
+    step = step_fused if fused else step_three
 
     def barrier():
         if world > 1:
@@ -276,10 +296,30 @@ def run_ours(args, cfg):
     ms_step = ms_total / args.steps
     value = world * flops / (ms_step * 1e-3) / 1e12
     att_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(ev["a0"], ev["a1"]))
-    reo_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(ev["r0"], ev["r1"])) / 3.0
-    uno_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(ev["u0"], ev["u1"]))
     if sta.sta_check_device_status(stream) != sta.STA_OK:
         raise RuntimeError("a kernel gave up on a bounded wait during timing")
+
+    # ---- the three-call path, for its per-kernel figures (not part of `value`)
+    ev3 = {n: [] for n in ("r0", "r1", "a0", "a1", "u0", "u1")}
+    three = None
+    if args.aux_steps > 0:
+        for _ in range(2):
+            step_three(False)
+        torch.cuda.synchronize()
+        for _ in range(args.aux_steps):
+            step_three(True, ev3)
+        torch.cuda.synchronize()
+        reo_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(ev3["r0"], ev3["r1"])) / 3.0
+        uno_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(ev3["u0"], ev3["u1"]))
+        att3_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(ev3["a0"], ev3["a1"]))
+        hbm = load_peaks().get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"])
+        reo_gbs = 2 * tensor_bytes / (reo_ms * 1e-3) / 1e9
+        three = {"steps": args.aux_steps, "step_ms": 3 * reo_ms + att3_ms + uno_ms,
+                 "tiled_attention_ms": att3_ms, "tiled_attention_tflops": flops / (att3_ms * 1e-3) / 1e12,
+                 "reorder_ms_per_tensor": reo_ms, "reorder_gbs": reo_gbs, "reorder_frac_hbm": reo_gbs / hbm,
+                 "unorder_ms": uno_ms, "unorder_gbs": 2 * tensor_bytes / (uno_ms * 1e-3) / 1e9}
+        if sta.sta_check_device_status(stream) != sta.STA_OK:
+            raise RuntimeError("a kernel gave up on a bounded wait during the three-call steps")
 
     # ---- end to end through the public API with host buffers
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
@@ -292,7 +332,7 @@ def run_ours(args, cfg):
         q.copy_(q_h, non_blocking=True)
         k.copy_(k_h, non_blocking=True)
         v.copy_(v_h, non_blocking=True)
-        o = sta.sta_forward(q, k, v, grid, tile, wins, scale, stream, workspace=ws)
+        o = sta.sta_forward(q, k, v, grid, tile, wins, scale, stream, workspace=ws, fused=fused)
         out_h.copy_(o, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
@@ -310,7 +350,6 @@ def run_ours(args, cfg):
     traffic = None
     if cfg.name == PROFILED_TRAFFIC["workload"] and kernel_source_sha1() == PROFILED_TRAFFIC["sha1"]:
         traffic = PROFILED_TRAFFIC["bytes_per_launch"]
-    reo_gbs = 2 * tensor_bytes / (reo_ms * 1e-3) / 1e9
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -323,19 +362,21 @@ def run_ours(args, cfg):
         "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(cfg, args),
-        "roofline": {"bound": "tensor", "kernel": "sta_fwd_kernel", "achieved": att_tflops, "peak": peak_s,
+        "roofline": {"bound": "tensor", "kernel": "sta_fwd_kernel" + ("<raster>" if fused else "<tiled>"),
+                     "achieved": att_tflops, "peak": peak_s,
                      "unit": "TFLOP/s", "frac": att_tflops / peak_s, "traffic": traffic,
                      "peak_kind": f"bf16_tflops_sustained ({peaks['_source']})",
                      "frac_of_burst_peak": att_tflops / peak_b, "frac_of_2250_datasheet": att_tflops / 2250.0},
         "kernels": {"attention_ms": att_ms, "attention_tflops": att_tflops,
-                    "reorder_ms_per_tensor": reo_ms, "reorder_gbs": reo_gbs, "reorder_frac_hbm": reo_gbs / hbm,
-                    "unorder_ms": uno_ms, "unorder_gbs": 2 * tensor_bytes / (uno_ms * 1e-3) / 1e9},
+                    "path": "fused raster-order kernel, 1 launch per step" if fused else
+                            "reorder x3 + tiled attention + unorder, 5 launches per step",
+                    "three_call_path": three},
         "cpu_baseline": cpu,
         "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": 3 * tensor_bytes, "d2h_bytes_per_step": tensor_bytes,
                 "steps": e2e_steps},
         "clocks": clk.summary(),
-        "gpu_launches": 5 * args.steps,
+        "gpu_launches": (1 if fused else 5) * args.steps,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -355,6 +396,10 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=4096)
     ap.add_argument("--ref-rows", type=int, default=512)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--three-call", action="store_true",
+                    help="time the reorder + tiled attention + unorder path as the step")
+    ap.add_argument("--aux-steps", type=int, default=10,
+                    help="extra steps of the three-call path for its per-kernel figures (0: none)")
     ap.add_argument("--heads", type=int, default=0,
                     help="use only the first N heads of the workload (small profiling cases)")
     args = ap.parse_args()

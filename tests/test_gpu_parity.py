@@ -213,11 +213,12 @@ def test_attention_perhead_sampled():
 def test_attention_score_jumps_exercise_rescale_paths():
     """Planted keys whose scores jump far above the running max in a later block.
 
-    Blocks after an item's first use the running max of the earlier blocks; a jump
-    of more than 2^64 takes the slow paths (first or second half of a block), smaller
-    jumps the deferred rescale.  Two query rows of an interior tile get one planted
-    key each, inside their own tile (never the first block of the window), one in
-    the first 64 keys of a 128-key block and one in the last 64.
+    The kernel moves a row's running max only when a block's max exceeds it by more
+    than 2^8, and then rescales O and the row sum together.  Random N(0, 1) inputs
+    never get there.  Two query rows of an interior tile get one planted key each,
+    scoring about 110 (log2 units) above the rest, inside their own tile (never the
+    first block of the window): one in the first 64 keys of a 128-key block and one
+    in the last 64.
     """
     cfg = W.custom_config("jumps", 1, 1, 128, (12, 24, 40), (6, 8, 8), [(1, 3, 3)])
     q, k, v = W.make_qkv(cfg, 11)
