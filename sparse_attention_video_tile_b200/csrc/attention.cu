@@ -6,32 +6,38 @@
 // innovation"), and the kernel is built around asynchronous loads and block
 // management (summary page, "AI overview").  On B200 that becomes:
 //
-//   * a persistent grid of one CTA per SM; each CTA runs two lanes, each lane a
-//     block of 128 query rows (one work item of the host window enumerator) at a
-//     time;
-//   * warp 8, the producer, streams each lane's Q once per item and then only
-//     the key and value blocks of the lane's window into a four-stage shared
-//     memory ring with TMA (128-byte swizzle, completion on mbarriers);
-//   * warp 9 issues every tcgen05 MMA from one thread: S = Q K^T (both operands
-//     in shared memory, fp32 accumulator in TMEM) and O += P V (P read from TMEM
-//     where it overwrote S, V from shared memory, O in TMEM);
-//   * warps 0-3 (lane 0) and 4-7 (lane 1), one query row per thread, TMEM lane
-//     = row, run the online softmax in fp32: row max, p = 2^(s*scale*log2e - m),
-//     row sum, P rounded to bf16 and written back to TMEM; O is rescaled only
-//     when the running max grows by more than 2^8 (the result is unchanged: O
-//     and the row sum always carry the same factor); the epilogue divides by the
-//     row sum and writes bf16 rows.
+//   * a persistent grid of one CTA per SM; a CTA works on one block of 128 query
+//     rows (one work item of the host window enumerator) at a time, and walks
+//     the key blocks of all its items as one stream;
+//   * warp 8, the producer, loads each item's Q (two buffers, so the next item's
+//     Q arrives early) and the key and value blocks of the windows into a shared
+//     memory ring with TMA (128-byte swizzle, completion on mbarriers), in the
+//     order the MMA issuers consume them;
+//   * warp 10 issues S = Q K^T (both operands in shared memory, fp32
+//     accumulator in TMEM) and warp 9 O += P V (P read from TMEM where it
+//     overwrote S, V from shared memory, O in TMEM), one thread each: an MMA
+//     issue returns at the tensor core's execution rate, so one issuer's
+//     barrier waits and commits are covered by the other's MMAs.  S has three
+//     TMEM buffers: S of block g+3 is issued as soon as P V of block g has
+//     read P from its buffer, so the scores of the next two blocks are ready
+//     while the softmax works on block g;
+//   * warps 0-7 run the online softmax in fp32, two warps per row: TMEM lane =
+//     query row, warp w and w+4 take key columns 0-63 and 64-127 of the rows of
+//     TMEM lane quadrant w.  Each loads the whole score row for the row max
+//     (no exchange needed), computes p = 2^(s*scale*log2e - m) for its half,
+//     keeps its half of the row sum, and writes its half of P (bf16) over the
+//     first columns of its half of S.  O is rescaled only when the running max
+//     grows by more than 2^8 (O and the row sum always carry the same factor, so
+//     O / l is unchanged); the epilogue adds the two half sums, divides and
+//     writes bf16 rows, each warp half of the head dimension.
 //
-// The producer and the MMA issuer walk the same fixed sequence of turns,
-// alternating lanes: a turn issues a lane's P*V for block j and its Q*K^T for
-// block j+1.  The tensor core therefore always has the other lane's work queued
-// while one lane's softmax runs (ping-pong), and the load order equals the
-// consumption order, so one ring serves both lanes.
-//
-// With Ntile a multiple of 128 no element mask exists at all.  Otherwise
-// (small tiles, ragged tails) the softmax masks whole key tiles outside the
-// row's window and keys past L.  Every wait is bounded (see ptx.cuh): a stuck
-// pipeline records an error code and the CTA drains and exits.
+// Every barrier that is waited on with a parity can never run two phases ahead
+// of its waiter (the per-buffer S, P and P*V barriers, the Q pair, the ring).
+// With Ntile a multiple of 128 no element mask exists at all.  Otherwise (small
+// tiles, ragged tails) the softmax masks whole key tiles outside the row's
+// window and keys past L; padded latents mask the pad keys of boundary blocks.
+// Every wait is bounded (see ptx.cuh): a stuck pipeline records an error code
+// and the CTA drains and exits.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -50,21 +56,14 @@ namespace {
 
 using namespace ptx;
 
-constexpr int kLanes = 2;
-constexpr int kThreads = 384;       // warps 0-3 / 4-7 softmax of lane 0 / 1, 8-9 producers, 10-11 MMA issuers
-constexpr int kProducerWarp0 = 8;   // + lane
-constexpr int kMmaWarp0 = 10;       // + lane; warp 10 also owns the TMEM allocation
-constexpr int kStages = 2;          // per-lane key/value ring stages (K_j, V_j, K_j+1, ... in order)
-constexpr int kTmemCols = 512;      // lane l: S at 256 l, O at 256 l + 128
+constexpr int kThreads = 352;       // warps 0-7 softmax + epilogue, 8 producer, 9-10 MMA issuers
+constexpr int kProducerWarp = 8;
+constexpr int kPvWarp = 9;          // issues O += P V; also owns the TMEM allocation
+constexpr int kSWarp = 10;          // issues S = Q K^T
+constexpr int kSBufs = 3;           // score buffers in TMEM
+constexpr int kTmemCols = 512;      // S buffer b at 128 b, O at kOCol
+constexpr int kOCol = 128 * kSBufs;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
-// Register split: launched at 168 per thread (384 threads, one CTA per SM);
-// the two softmax warpgroups take 208 each, the producer/MMA warpgroup keeps 88:
-// 2 * 128 * 208 + 128 * 88 = 384 * 168.
-constexpr int kLaunchRegs = 168;
-constexpr int kRegsSoftmax = 208;
-constexpr int kRegsOther = 88;
-static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsOther == kThreads * kLaunchRegs,
-              "register split must match the launch");
 constexpr int kDefaultPoly8 = 0;
 
 struct FwdParams {
@@ -73,7 +72,7 @@ struct FwdParams {
   const int32_t* kv_mask_id; // per kv_rows entry: -1 or a key-validity mask (padded latents), or null
   const uint32_t* kv_masks;  // 4 words per mask
   const int16_t* head_win;   // [heads][4]
-  __nv_bfloat16* out;        // [BH, L, d] tiled order
+  __nv_bfloat16* out;        // [BH, L, d] tiled order, or raster order
   int32_t n_items;
   int32_t heads;
   int32_t L;
@@ -88,27 +87,31 @@ struct FwdParams {
 
 template <int D>
 struct Smem {
+  static constexpr int kQBufs = 2;                         // Q buffers (item k in buffer k mod kQBufs)
+  static constexpr int kStages = D == 64 ? 8 : 4;          // key/value ring stages
   static constexpr int kBlockBytes = kBlockRows * D * 2;  // one 128-row block of Q, K or V
-  static constexpr int kQ0 = 0;                            // lane l's Q at kQ0 + l * kBlockBytes
-  static constexpr int kStage0 = kLanes * kBlockBytes;     // lane l's stage s at kStage0 + (l * kStages + s) * kBlockBytes
-  static constexpr int kBar = kStage0 + kLanes * kStages * kBlockBytes;
-  // per-lane barriers (8 bytes each), lane l's copy at + l * kBarStride
-  static constexpr int kQFull = 0;
-  static constexpr int kQEmpty = 8;
-  static constexpr int kKvFull = 16;                       // [stage]
+  static constexpr int kQ = 0;                             // Q buffer b at kQ + b * kBlockBytes
+  static constexpr int kStage0 = kQBufs * kBlockBytes;     // stage s at kStage0 + s * kBlockBytes
+  static constexpr int kLx = kStage0 + kStages * kBlockBytes;  // float [item parity][half][row]
+  static constexpr int kBar = kLx + 2 * 2 * kBlockRows * 4;
+  static constexpr int kQFull = kBar;                      // [Q buffer]
+  static constexpr int kQEmpty = kQFull + 16;              // [Q buffer]
+  static constexpr int kKvFull = kQEmpty + 16;             // [stage]
   static constexpr int kKvEmpty = kKvFull + 8 * kStages;   // [stage]
-  static constexpr int kSFull = kKvEmpty + 8 * kStages;
-  static constexpr int kPLo = kSFull + 8;                  // P of keys 0-63 written
-  static constexpr int kPHi = kPLo + 8;                    // P of keys 64-127 written
-  static constexpr int kOFull = kPHi + 8;
+  static constexpr int kSFull = kKvEmpty + 8 * kStages;    // [S buffer]: S written
+  static constexpr int kPFull = kSFull + 8 * kSBufs;       // [S buffer]: P written (8 warps)
+  static constexpr int kPvDone = kPFull + 8 * kSBufs;      // [S buffer]: P V of that block completed
+  static constexpr int kSRead = kPvDone + 8 * kSBufs;      // [lane quadrant]: both warps hold S
+  static constexpr int kLxBar = kSRead + 8 * 4;            // [lane quadrant]: half row sums written
+  static constexpr int kOFull = kLxBar + 8 * 4;
   static constexpr int kDrain = kOFull + 8;
-  static constexpr int kTurn = kDrain + 8;                 // this lane may run its exponentials
-  static constexpr int kBarStride = kTurn + 8;
-  static constexpr int kTmemSlot = kBar + kLanes * kBarStride;
+  static constexpr int kDrainS = kDrain + 8;
+  static constexpr int kTmemSlot = kDrainS + 8;
   static constexpr int kAbort = kTmemSlot + 4;
   static constexpr int kEnd = kAbort + 4;
   static constexpr int kDynBytes = kEnd + 1024;  // + slack to align the base to 1024
   static_assert(kDynBytes <= 227 * 1024, "shared memory budget");
+  static_assert(kBlockBytes % 1024 == 0, "swizzled tiles need 1024-byte alignment");
 };
 
 // TMA coordinates (x, w, h, t) of the 128-row slab that starts at tiled row
@@ -123,17 +126,41 @@ __device__ __forceinline__ SlabCoord slab_coord(const FwdParams& p, int32_t row)
   return SlabCoord{aw * p.tw, ah * p.th, at * p.tt + b * p.bt};
 }
 
-// Item k of lane l of CTA c is (k * gridDim.x + c) * 2 + l: at any time the CTAs
-// work on adjacent items (neighbouring query blocks, overlapping windows).
-__device__ __forceinline__ int32_t lane_item(int32_t k, int lane) {
-  return (k * static_cast<int32_t>(gridDim.x) + static_cast<int32_t>(blockIdx.x)) * kLanes + lane;
-}
+// Position in the stream of key blocks of this CTA: item ordinal k (item index
+// k * gridDim.x + blockIdx.x; neighbouring CTAs work on neighbouring items, whose
+// windows overlap in L2), block j of that item, and g, the block's ordinal over
+// all the CTA's items.
+struct BlockCursor {
+  int32_t k, j, g;
+  WorkItem it;
+  bool done;
+  __device__ __forceinline__ void load(const FwdParams& p) {
+    const int32_t idx = k * static_cast<int32_t>(gridDim.x) + static_cast<int32_t>(blockIdx.x);
+    done = idx >= p.n_items;
+    if (!done) it = p.items[idx];
+  }
+  __device__ __forceinline__ void start(const FwdParams& p) {
+    k = 0;
+    j = 0;
+    g = 0;
+    load(p);
+  }
+  __device__ __forceinline__ void next(const FwdParams& p) {
+    ++g;
+    if (++j == it.kv_len) {
+      j = 0;
+      ++k;
+      load(p);
+    }
+  }
+};
 
 template <int D, bool MASKED, int POLY8, bool RASTER>
 __global__ void __launch_bounds__(kThreads, 1)
     sta_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
   using S = Smem<D>;
+  constexpr int kStages = S::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
@@ -144,25 +171,30 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::kTmemSlot);
 
   if (threadIdx.x == 0) {
-    for (int l = 0; l < kLanes; ++l) {
-      const uint32_t b = sb + S::kBar + l * S::kBarStride;
-      mbar_init(b + S::kQFull, 1);
-      mbar_init(b + S::kQEmpty, 1);
-      for (int s = 0; s < kStages; ++s) {
-        mbar_init(b + S::kKvFull + 8 * s, 1);
-        mbar_init(b + S::kKvEmpty + 8 * s, 1);
-      }
-      mbar_init(b + S::kSFull, 1);
-      mbar_init(b + S::kPLo, 4);   // one arrival per softmax warp
-      mbar_init(b + S::kPHi, 4);
-      mbar_init(b + S::kOFull, 1);
-      mbar_init(b + S::kDrain, 1);
-      mbar_init(b + S::kTurn, 4);
+    for (int b = 0; b < S::kQBufs; ++b) {
+      mbar_init(sb + S::kQFull + 8 * b, 1);
+      mbar_init(sb + S::kQEmpty + 8 * b, 1);
     }
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(sb + S::kKvFull + 8 * s, 1);
+      mbar_init(sb + S::kKvEmpty + 8 * s, 1);
+    }
+    for (int b = 0; b < kSBufs; ++b) {
+      mbar_init(sb + S::kSFull + 8 * b, 1);
+      mbar_init(sb + S::kPFull + 8 * b, 8);    // one arrival per softmax warp
+      mbar_init(sb + S::kPvDone + 8 * b, 1);
+    }
+    for (int q = 0; q < 4; ++q) {
+      mbar_init(sb + S::kSRead + 8 * q, 2);    // one arrival per warp of the pair
+      mbar_init(sb + S::kLxBar + 8 * q, 64);   // every thread of the pair
+    }
+    mbar_init(sb + S::kOFull, 1);
+    mbar_init(sb + S::kDrain, 1);
+    mbar_init(sb + S::kDrainS, 1);
     *abort_flag = 0;
     fence_mbarrier_init();
   }
-  if (warp == kMmaWarp0) {
+  if (warp == kPvWarp) {
     tmem_alloc(sb + S::kTmemSlot, kTmemCols);
     tmem_relinquish();
   }
@@ -176,179 +208,171 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int kBoxes = D / 64;
   constexpr uint32_t kBlockBytes = S::kBlockBytes;
 
-  if (warp == kProducerWarp0 || warp == kProducerWarp0 + 1) {
-    // ------------------------------------------------------------ producer of one lane
-    setmaxnreg_dec<kRegsOther>();
-    const int ln = warp - kProducerWarp0;
+  if (warp == kProducerWarp) {
+    // ------------------------------------------------------------ producer
     if (lane == 0) {
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
-      const uint32_t bars = sb + S::kBar + ln * S::kBarStride;
-      const uint32_t qdst = sb + S::kQ0 + ln * kBlockBytes;
-      const uint32_t ring = sb + S::kStage0 + ln * kStages * kBlockBytes;
-      uint32_t kv_seq = 0, q_loads = 0;
+      uint32_t kv_seq = 0, q_loads[2] = {0, 0};
       bool ok = true;
-      // one key or value block into the lane's next ring stage
-      auto load_block = [&](const CUtensorMap* m, int32_t row, int32_t bh) -> bool {
-        const uint32_t st = kv_seq % kStages;
-        if (!mbar_wait(bars + S::kKvEmpty + 8 * st, ((kv_seq / kStages) & 1) ^ 1, wc, 2)) return false;
-        const uint32_t dst = ring + st * kBlockBytes;
-        const uint32_t full = bars + S::kKvFull + 8 * st;
-        mbar_arrive_expect_tx(full, kBlockBytes);
+      // one 128-row block (Q into buffer `dst`, or K/V into the next ring stage)
+      auto tma_block = [&](uint32_t dst, const CUtensorMap* m, uint32_t full, int32_t row, int32_t bh) {
         if constexpr (RASTER) {
           const SlabCoord c = slab_coord(p, row);
           for (int b = 0; b < kBoxes; ++b) tma_load_5d(dst + b * kBoxBytes, m, full, b * 64, c.w, c.h, c.t, bh);
         } else {
           for (int b = 0; b < kBoxes; ++b) tma_load_3d(dst + b * kBoxBytes, m, full, b * 64, row, bh);
         }
+      };
+      auto load_ring = [&](const CUtensorMap* m, int32_t row, int32_t bh) -> bool {
+        const uint32_t st = kv_seq % kStages;
+        if (!mbar_wait(sb + S::kKvEmpty + 8 * st, ((kv_seq / kStages) & 1) ^ 1, wc, 2)) return false;
+        const uint32_t full = sb + S::kKvFull + 8 * st;
+        mbar_arrive_expect_tx(full, kBlockBytes);
+        tma_block(sb + S::kStage0 + st * kBlockBytes, m, full, row, bh);
         ++kv_seq;
         return true;
       };
-      for (int32_t k = 0; ok; ++k) {
-        const int32_t idx = lane_item(k, ln);
-        if (idx >= p.n_items) break;
-        const WorkItem item = p.items[idx];
-        ok = mbar_wait(bars + S::kQEmpty, (q_loads & 1) ^ 1, wc, 1);
-        if (!ok) break;
-        ++q_loads;
-        mbar_arrive_expect_tx(bars + S::kQFull, kBlockBytes);
-        if constexpr (RASTER) {
-          const SlabCoord c = slab_coord(p, item.q_row0);
-          for (int b = 0; b < kBoxes; ++b)
-            tma_load_5d(qdst + b * kBoxBytes, &tm_q, bars + S::kQFull, b * 64, c.w, c.h, c.t, item.bh);
-        } else {
-          for (int b = 0; b < kBoxes; ++b)
-            tma_load_3d(qdst + b * kBoxBytes, &tm_q, bars + S::kQFull, b * 64, item.q_row0, item.bh);
+      // K of block (k, j), preceded by the item's Q when j = 0
+      auto load_k = [&](const BlockCursor& c) -> bool {
+        if (c.j == 0) {
+          const int qb = c.k % S::kQBufs;
+          if (!mbar_wait(sb + S::kQEmpty + 8 * qb, ((c.k / S::kQBufs) & 1) ^ 1, wc, 1)) return false;
+          mbar_arrive_expect_tx(sb + S::kQFull + 8 * qb, kBlockBytes);
+          tma_block(sb + S::kQ + qb * kBlockBytes, &tm_q, sb + S::kQFull + 8 * qb, c.it.q_row0, c.it.bh);
+          ++q_loads[qb];
         }
-        for (int32_t j = 0; j < item.kv_len && ok; ++j) {
-          const int32_t row = p.kv_rows[item.kv_off + j];
-          ok = load_block(&tm_k, row, item.bh) && load_block(&tm_v, row, item.bh);
+        return load_ring(&tm_k, p.kv_rows[c.it.kv_off + c.j], c.it.bh);
+      };
+      // Order of the loads: K_0, K_1, K_2, then V_g, K_g+3 for g = 0, 1, ... (the S
+      // issuer needs K three blocks ahead of the P V issuer's V).
+      BlockCursor kc, vc;
+      kc.start(p);
+      vc.start(p);
+      for (int i = 0; i < kSBufs && ok && !kc.done; ++i) {
+        ok = load_k(kc);
+        kc.next(p);
+      }
+      while (ok && !vc.done) {
+        ok = load_ring(&tm_v, p.kv_rows[vc.it.kv_off + vc.j], vc.it.bh);
+        vc.next(p);
+        if (ok && !kc.done) {
+          ok = load_k(kc);
+          kc.next(p);
         }
       }
       // Drain: every load issued has landed before the CTA may exit.  Waiting on a
       // phase that already completed returns at once.
-      if (q_loads > 0) mbar_wait_drain(bars + S::kQFull, (q_loads - 1) & 1, p.limit_ns);
+      for (int b = 0; b < S::kQBufs; ++b)
+        if (q_loads[b] > 0) mbar_wait_drain(sb + S::kQFull + 8 * b, (q_loads[b] - 1) & 1, p.limit_ns);
       for (uint32_t s = 0; s < kStages && s < kv_seq; ++s) {
         const uint32_t last = kv_seq - 1 - ((kv_seq - 1 - s) % kStages);  // last sequence number on stage s
-        mbar_wait_drain(bars + S::kKvFull + 8 * s, (last / kStages) & 1, p.limit_ns);
+        mbar_wait_drain(sb + S::kKvFull + 8 * s, (last / kStages) & 1, p.limit_ns);
       }
     }
     __syncwarp();
-  } else if (warp == kMmaWarp0 || warp == kMmaWarp0 + 1) {
-    // ------------------------------------------------------------ MMA issuer of one lane
-    setmaxnreg_dec<kRegsOther>();
-    const int ln = warp - kMmaWarp0;
+  } else if (warp == kPvWarp || warp == kSWarp) {
+    // ------------------------------------------------------------ MMA issuers
+    // A tcgen05.mma issue returns at about the rate the tensor core executes, so
+    // whatever else an issuing thread does (barrier waits, commits, bookkeeping)
+    // leaves the tensor core idle unless another thread is issuing meanwhile: S
+    // and P*V have one issuer each.
     if (lane == 0) {
-      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
-      const uint32_t bars = sb + S::kBar + ln * S::kBarStride;
-      const uint32_t tS = tmem + 256 * ln, tO = tS + 128;
       // Shared-memory descriptors differ only in the start-address field (bits 0-13,
       // address >> 4; every address here is below 256 KB, so adding an offset never
       // carries out of the field): one base descriptor per role plus offsets.
-      const uint64_t dq = sdesc_sw128(sb + S::kQ0 + ln * kBlockBytes, 16, 1024);        // K-major (Q)
-      const uint32_t ring = sb + S::kStage0 + ln * kStages * kBlockBytes;
-      const uint64_t dk0 = sdesc_sw128(ring, 16, 1024);                                   // K-major (K)
-      const uint64_t dv0 = sdesc_sw128(ring, kBlockRows * 128, 1024);                     // MN-major (V)
-      constexpr uint32_t kStageStep = kBlockBytes >> 4;
-      // slice k16 of a K-major block: 64-column boxes of 16 KB, 32 bytes per 16 columns
-      auto koff = [](int k16) -> uint64_t { return static_cast<uint64_t>(((k16 >> 2) * 16384 + (k16 & 3) * 32) >> 4); };
-      auto wait_stage = [&](uint32_t seq, int site) -> bool {
-        return mbar_wait(bars + S::kKvFull + 8 * (seq % kStages), (seq / kStages) & 1, wc, site);
-      };
-      // S = Q K^T from ring stage st
-      auto issue_qk = [&](uint32_t st) {
-        const uint64_t dk = dk0 + st * kStageStep;
-#pragma unroll
-        for (int k16 = 0; k16 < D / 16; ++k16)
-          umma_ss(tS, dq + koff(k16), dk + koff(k16), idesc_qk, k16 > 0 ? 1u : 0u);
-        umma_commit(bars + S::kKvEmpty + 8 * st);
-      };
-      // O += P V for keys [64 h, 64 h + 64) of ring stage st (16 keys = 2 KB per slice)
-      auto issue_pv_half = [&](uint32_t st, int h, bool accumulate) {
-        const uint64_t dv = dv0 + st * kStageStep;
-#pragma unroll
-        for (int k16 = 4 * h; k16 < 4 * h + 4; ++k16)
-          umma_ts(tO, tS + k16 * 8, dv + static_cast<uint64_t>(k16 * (2048 >> 4)), idesc_pv,
-                  (accumulate || k16 > 0) ? 1u : 0u);
-      };
-      uint32_t kv_seq = 0, p_waits = 0;
-      bool ok = true;
-      for (int32_t k = 0; ok; ++k) {
-        const int32_t idx = lane_item(k, ln);
+      constexpr uint32_t kBlockStep = kBlockBytes >> 4;
+      // Ring sequence numbers of the loads, in the producer's order K_0, K_1, K_2,
+      // V_0, K_3, V_1, ...: K_g is load g + max(0, g - 2) and V_g is load
+      // min(G + g, 2 g + 3), G being the number of blocks of this CTA.
+      int32_t G = 0;
+      for (int32_t k = 0;; ++k) {
+        const int32_t idx = k * static_cast<int32_t>(gridDim.x) + static_cast<int32_t>(blockIdx.x);
         if (idx >= p.n_items) break;
-        const int32_t n = p.items[idx].kv_len;
-        ok = mbar_wait(bars + S::kQFull, k & 1, wc, 3) && wait_stage(kv_seq, 4);
-        if (!ok) break;
-        tc_fence_after();
-        issue_qk(kv_seq % kStages);  // S_0
-        ++kv_seq;
-        if (n == 1) umma_commit(bars + S::kQEmpty);
-        umma_commit(bars + S::kSFull);
-        for (int32_t j = 0; j < n && ok; ++j) {
-          // V_j and K_j+1 were loaded ahead: wait for them first, so that only the
-          // softmax hand-off (P_j) stands between S_j and these MMAs.
-          const bool has_k = j + 1 < n;
-          ok = wait_stage(kv_seq, 6) && (!has_k || wait_stage(kv_seq + 1, 4)) &&
-               mbar_wait(bars + S::kPLo, p_waits & 1, wc, 5);
+        G += p.items[idx].kv_len;
+      }
+      auto wait_load = [&](uint32_t seq, int site) -> bool {
+        return mbar_wait(sb + S::kKvFull + 8 * (seq % kStages), (seq / kStages) & 1, wc, site);
+      };
+      BlockCursor c;
+      c.start(p);
+      bool ok = true;
+      if (warp == kSWarp) {
+        // S_g = Q K_g^T into S buffer g mod 3, once P_g-3 V_g-3 (which reads P_g-3
+        // from that buffer) has completed.
+        constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
+        const uint64_t dq0 = sdesc_sw128(sb + S::kQ, 16, 1024);                         // K-major (Q)
+        const uint64_t dk0 = sdesc_sw128(sb + S::kStage0, 16, 1024);                    // K-major (K)
+        // slice k16 of a K-major block: 64-column boxes of 16 KB, 32 bytes per 16 columns
+        auto koff = [](int k16) -> uint64_t { return static_cast<uint64_t>(((k16 >> 2) * 16384 + (k16 & 3) * 32) >> 4); };
+        for (; ok && !c.done; c.next(p)) {
+          const int32_t g = c.g;
+          const int b = g % kSBufs;
+          const int qb = c.k % S::kQBufs;
+          const uint32_t seq = static_cast<uint32_t>(g + (g > 2 ? g - 2 : 0));
+          ok = (g < kSBufs || mbar_wait(sb + S::kPvDone + 8 * b, ((g / kSBufs) & 1) ^ 1, wc, 14)) &&
+               (c.j != 0 || mbar_wait(sb + S::kQFull + 8 * qb, (c.k / S::kQBufs) & 1, wc, 3)) && wait_load(seq, 4);
           if (!ok) break;
           tc_fence_after();
-          // O += P_j V_j, the first 64 keys as soon as their P is written
-          issue_pv_half(kv_seq % kStages, 0, j > 0);
-          ok = mbar_wait(bars + S::kPHi, p_waits & 1, wc, 10);
-          ++p_waits;
-          if (!ok) break;
-          tc_fence_after();
-          issue_pv_half(kv_seq % kStages, 1, true);
-          umma_commit(bars + S::kKvEmpty + 8 * (kv_seq % kStages));
-          ++kv_seq;
-          if (has_k) {
-            issue_qk(kv_seq % kStages);  // S_j+1 (overwrites P_j after P_j V_j, in issue order)
-            ++kv_seq;
-            if (j + 2 == n) umma_commit(bars + S::kQEmpty);
-            umma_commit(bars + S::kSFull);
-          }
+          const uint32_t st = seq % kStages;
+          const uint64_t dq = dq0 + qb * kBlockStep, dk = dk0 + st * kBlockStep;
+#pragma unroll
+          for (int k16 = 0; k16 < D / 16; ++k16)
+            umma_ss(tmem + 128 * b, dq + koff(k16), dk + koff(k16), idesc_qk, k16 > 0 ? 1u : 0u);
+          umma_commit(sb + S::kKvEmpty + 8 * st);
+          if (c.j + 1 == c.it.kv_len) umma_commit(sb + S::kQEmpty + 8 * qb);
+          umma_commit(sb + S::kSFull + 8 * b);
         }
-        if (ok) umma_commit(bars + S::kOFull);
+      } else {
+        // O += P_g V_g: keys 0-63 with P in S columns 0-31, keys 64-127 with P in
+        // S columns 64-95 (16 keys = 8 columns of P, 2 KB of V per slice)
+        constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
+        const uint32_t tO = tmem + kOCol;
+        const uint64_t dv0 = sdesc_sw128(sb + S::kStage0, kBlockRows * 128, 1024);      // MN-major (V)
+        for (; ok && !c.done; c.next(p)) {
+          const int32_t g = c.g;
+          const int b = g % kSBufs;
+          const uint32_t seq = static_cast<uint32_t>(min(G + g, 2 * g + 3));
+          ok = wait_load(seq, 6) && mbar_wait(sb + S::kPFull + 8 * b, (g / kSBufs) & 1, wc, 5);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t st = seq % kStages;
+          const uint64_t dv = dv0 + st * kBlockStep;
+          const uint32_t tP = tmem + 128 * b;
+#pragma unroll
+          for (int k16 = 0; k16 < 8; ++k16)
+            umma_ts(tO, tP + (k16 >> 2) * 64 + (k16 & 3) * 8, dv + static_cast<uint64_t>(k16 * (2048 >> 4)), idesc_pv,
+                    (c.j > 0 || k16 > 0) ? 1u : 0u);
+          umma_commit(sb + S::kKvEmpty + 8 * st);
+          umma_commit(sb + S::kPvDone + 8 * b);
+          if (c.j + 1 == c.it.kv_len) umma_commit(sb + S::kOFull);
+        }
       }
       // Drain: all MMAs issued by this thread complete before TMEM is freed.
-      umma_commit(bars + S::kDrain);
-      mbar_wait_drain(bars + S::kDrain, 0, p.limit_ns);
+      const uint32_t drain = sb + (warp == kSWarp ? S::kDrainS : S::kDrain);
+      umma_commit(drain);
+      mbar_wait_drain(drain, 0, p.limit_ns);
     }
     __syncwarp();
-  } else if (warp < 8) {
+  } else {
     // ------------------------------------------------------------ softmax + epilogue
-    setmaxnreg_inc<kRegsSoftmax>();
-    const int ln = warp >> 2;                             // this warpgroup's lane
-    const int row = threadIdx.x & 127;                    // TMEM lane = query row in the block
-    const uint32_t trow = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16) + 256 * ln;
-    const uint32_t tS = trow, tO = trow + 128;
-    const uint32_t bars = sb + S::kBar + ln * S::kBarStride;
-    const uint32_t bar_s = bars + S::kSFull, bar_plo = bars + S::kPLo, bar_phi = bars + S::kPHi,
-                   bar_o = bars + S::kOFull;
+    const int h = warp >> 2;                              // key columns [64 h, 64 h + 64)
+    const int quad = warp & 3;                            // TMEM lane quadrant
+    const int row = quad * 32 + lane;                     // TMEM lane = query row in the block
+    const uint32_t tlane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    const uint32_t tO = tlane + kOCol + h * (D / 2);      // this warp's half of O
+    const uint32_t bar_sread = sb + S::kSRead + 8 * quad, bar_lx = sb + S::kLxBar + 8 * quad;
+    float* lx = reinterpret_cast<float*>(smem + S::kLx);
     const float sl2 = p.scale_log2;
-    uint32_t sphase = 0, it = 0;
+    int32_t g = 0;
     bool ok = true;
-    // Turn token: the two lanes' exponential loops alternate (lane 0 block b after
-    // lane 1 block b-1, lane 1 block b after lane 0 block b) while both have blocks,
-    // so that each has the SM's MUFU units to itself and the other lane's MMAs run
-    // meanwhile.  A lane never gets more than one phase ahead, so parity waits are
-    // exact.
-    int32_t other_total = 0;
-    for (int32_t kk = 0;; ++kk) {
-      const int32_t oi = lane_item(kk, ln ^ 1);
-      if (oi >= p.n_items) break;
-      other_total += p.items[oi].kv_len;
-    }
-    const uint32_t my_turn = bars + S::kTurn;
-    const uint32_t their_turn = sb + S::kBar + (ln ^ 1) * S::kBarStride + S::kTurn;
-    for (int32_t k = 0; ok; ++k, ++it) {
-      const int32_t idx = lane_item(k, ln);
+    for (int32_t k = 0; ok; ++k) {
+      const int32_t idx = k * static_cast<int32_t>(gridDim.x) + static_cast<int32_t>(blockIdx.x);
       if (idx >= p.n_items) break;
       const WorkItem item = p.items[idx];
       float m_run = -INFINITY;
-      float l_run = 0.f;
+      float l_run = 0.f;   // this warp's half of the row sum
       // masked path: this row's window box in tile coordinates
       int32_t ws_t = 0, ws_h = 0, ws_w = 0, we_t = 0, we_h = 0, we_w = 0;
       if (MASKED) {
@@ -361,25 +385,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         ws_h = min(max(ah - eh / 2, 0), p.nH - eh); we_h = ws_h + eh;
         ws_w = min(max(aw - ew / 2, 0), p.nW - ew); we_w = ws_w + ew;
       }
-      for (int j = 0; j < item.kv_len; ++j) {
-        ok = __all_sync(0xffffffffu, mbar_wait(bar_s, sphase & 1, wc, 7));
-        const int32_t blk = static_cast<int32_t>(sphase);  // blocks of this lane before this one
-        ++sphase;
+      for (int j = 0; j < item.kv_len; ++j, ++g) {
+        const int b = g % kSBufs;
+        const uint32_t tS = tlane + 128 * b;
+        ok = __all_sync(0xffffffffu, mbar_wait(sb + S::kSFull + 8 * b, (g / kSBufs) & 1, wc, 7));
         if (!ok) break;
         tc_fence_after();
-        // The whole score row (128 fp32) in one round trip.
+        // The whole score row in one round trip: this warp's half into r[0, 64),
+        // the other half into r[64, 128) (for the row max only).
         uint32_t r[128];
-        tmem_ld32_at<0>(tS, r);
-        tmem_ld32_at<32>(tS + 32, r);
-        tmem_ld32_at<64>(tS + 64, r);
-        tmem_ld32_at<96>(tS + 96, r);
+        tmem_ld32_at<0>(tS + 64 * h, r);
+        tmem_ld32_at<32>(tS + 64 * h + 32, r);
+        tmem_ld32_at<64>(tS + 64 * (h ^ 1), r);
+        tmem_ld32_at<96>(tS + 64 * (h ^ 1) + 32, r);
         tmem_wait_ld();
+        // This warp holds S now: the other warp of the pair may overwrite its half with P.
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_sread);
+        // r[i] holds key column col(i) of the block
+        auto col = [h](int i) -> int { return i < 64 ? 64 * h + i : 64 * (h ^ 1) + (i - 64); };
         if (!MASKED && p.kv_mask_id != nullptr) {
           // padded latent: keys of pad tokens in this block do not exist
           const int32_t mid = p.kv_mask_id[item.kv_off + j];
           if (mid >= 0) {
             const uint4 mw = *reinterpret_cast<const uint4*>(p.kv_masks + 4 * mid);
-            const uint32_t words[4] = {mw.x, mw.y, mw.z, mw.w};
+            const uint32_t own0 = h ? mw.z : mw.x, own1 = h ? mw.w : mw.y;
+            const uint32_t oth0 = h ? mw.x : mw.z, oth1 = h ? mw.y : mw.w;
+            const uint32_t words[4] = {own0, own1, oth0, oth1};
 #pragma unroll
             for (int i = 0; i < 128; ++i)
               if (!((words[i >> 5] >> (i & 31)) & 1u)) r[i] = __float_as_uint(-INFINITY);
@@ -389,7 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int32_t kv_row = p.kv_rows[item.kv_off + j];
 #pragma unroll
           for (int i = 0; i < 128; ++i) {
-            const int32_t key = kv_row + i;
+            const int32_t key = kv_row + col(i);
             bool in = key < p.L;
             if (in) {
               const int32_t kt = key / p.ntile;
@@ -413,6 +446,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float m_blk = mx * sl2;
         // The running max moves only when it grows by more than 2^8: p stays <= 256
         // and O and the row sum always carry the same factor, so O / l is exact.
+        // Both warps of a row see the same scores, so they take the same decision.
         const bool need = (m_run != -INFINITY) && (m_blk > m_run + kRescaleThreshold);
         float f = 1.0f;
         if (m_run == -INFINITY) {
@@ -422,12 +456,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           l_run *= f;
           m_run = m_blk;
         }
-        // O (complete up to the previous block: its P*V finished before this S was
-        // committed) is rescaled by the whole warp when any of its rows needs it;
-        // tcgen05.ld/st are warp-collective.
         if (__any_sync(0xffffffffu, need)) {
+          // O holds P V up to block g-1, whose product may still be running: wait
+          // for it, then rescale this warp's half of O (tcgen05.ld/st are
+          // warp-collective, so the whole warp takes part).
+          const int pb = (g + kSBufs - 1) % kSBufs;
+          ok = __all_sync(0xffffffffu, mbar_wait(sb + S::kPvDone + 8 * pb, ((g - 1) / kSBufs) & 1, wc, 11));
+          if (!ok) break;
+          tc_fence_after();
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
+          for (int c = 0; c < D / 64; ++c) {
             uint32_t o[32];
             tmem_ld32(tO + c * 32, o);
             tmem_wait_ld();
@@ -437,60 +475,40 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         const float nm = (m_run == -INFINITY) ? 0.f : -m_run;
-        {
-          const int32_t need = ln == 0 ? blk - 1 : blk;  // the other lane's block to wait for
-          if (need >= 0 && need < other_total) {
-            ok = __all_sync(0xffffffffu, mbar_wait(my_turn, static_cast<uint32_t>(need & 1), wc, 9));
-            if (!ok) break;
-          }
-        }
-        // p = 2^(s * scale * log2e - m): POLY8 of every 8 column pairs on the FMA pipe,
-        // the rest on MUFU; partial row sums; P packed to bf16 pairs.  Each half
-        // of the row (64 keys) is stored and handed to the MMA issuer on its own, so
-        // P V of the first half overlaps the exponentials of the second.
-        // x = s * scale * log2e - m and the row sums use packed fp32 pairs (one
-        // instruction per two columns); four pair-accumulators break the add chain.
+        // p = 2^(s * scale * log2e - m) for this warp's 64 keys: POLY8 of every 8
+        // column pairs on the FMA pipe, the rest on MUFU; x and the row sums use
+        // packed fp32 pairs (one instruction per two columns); four
+        // pair-accumulators break the add chain; P packed to bf16 pairs.
         const uint64_t sl2x2 = f32x2(sl2, sl2), nmx2 = f32x2(nm, nm);
         uint64_t ls2[4] = {0, 0, 0, 0};
-        uint32_t pk[64];
+        uint32_t pk[32];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-#pragma unroll
-          for (int i = 64 * h; i < 64 * h + 64; i += 2) {
-            const uint64_t x2 = fma_f32x2(f32x2(SV(i), SV(i + 1)), sl2x2, nmx2);
-            float p0, p1;
-            if (!MASKED && ((i >> 1) & 7) >= 8 - POLY8) {
-              // x >= -125 is kept by the clamp below; x <= 8 by the rescale threshold
-              float x0, x1;
-              f32x2_split(x2, x0, x1);
-              exp2_poly3_pair(f32x2(fmaxf(x0, -125.f), fmaxf(x1, -125.f)), p0, p1);
-            } else {
-              float x0, x1;
-              f32x2_split(x2, x0, x1);
-              p0 = ex2_approx(x0);
-              p1 = ex2_approx(x1);
-            }
-            ls2[(i >> 1) & 3] = add_f32x2(ls2[(i >> 1) & 3], f32x2(p0, p1));
-            pk[i >> 1] = pack_bf16x2(p0, p1);
-          }
-          // Each warp publishes its P with one elected arrival once all its lanes'
-          // TMEM stores are complete (wait::st, fence before the warp sync).
-          if (h == 0) {
-            tmem_st32_at<0>(tS, pk);
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar_plo);
+        for (int i = 0; i < 64; i += 2) {
+          const uint64_t x2 = fma_f32x2(f32x2(SV(i), SV(i + 1)), sl2x2, nmx2);
+          float p0, p1;
+          float x0, x1;
+          f32x2_split(x2, x0, x1);
+          if (!MASKED && ((i >> 1) & 7) >= 8 - POLY8) {
+            // x >= -125 is kept by the clamp; x <= 8 by the rescale threshold
+            exp2_poly3_pair(f32x2(fmaxf(x0, -125.f), fmaxf(x1, -125.f)), p0, p1);
           } else {
-            if (lane == 0) mbar_arrive(their_turn);  // the other lane may start its exponentials
-            tmem_st32_at<32>(tS + 32, pk);
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar_phi);
+            p0 = ex2_approx(x0);
+            p1 = ex2_approx(x1);
           }
+          ls2[(i >> 1) & 3] = add_f32x2(ls2[(i >> 1) & 3], f32x2(p0, p1));
+          pk[i >> 1] = pack_bf16x2(p0, p1);
         }
 #undef SV
+        // P over the first 32 columns of this warp's half of S, once the other warp
+        // of the pair has its copy of S.
+        ok = __all_sync(0xffffffffu, mbar_wait(bar_sread, static_cast<uint32_t>(g) & 1, wc, 12));
+        if (!ok) break;
+        tc_fence_after();
+        tmem_st32_at<0>(tS + 64 * h, pk);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(sb + S::kPFull + 8 * b);
         {
           float a0, a1, b0, b1, c0, c1, d0, d1;
           f32x2_split(ls2[0], a0, a1);
@@ -501,20 +519,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (!ok) break;
-      // epilogue: O / l -> bf16 rows (tiled order)
-      ok = __all_sync(0xffffffffu, mbar_wait(bar_o, it & 1, wc, 8));
+      // epilogue: O / l -> bf16, this warp's half of the head dimension
+      ok = __all_sync(0xffffffffu, mbar_wait(sb + S::kOFull, static_cast<uint32_t>(k) & 1, wc, 8));
       if (!ok) break;
       tc_fence_after();
-      uint32_t o[D];
+      uint32_t o[D / 2];
       tmem_ld32_at<0>(tO, o);
-      tmem_ld32_at<32>(tO + 32, o);
-      if constexpr (D == 128) {
-        tmem_ld32_at<64>(tO + 64, o);
-        tmem_ld32_at<96>(tO + 96, o);
-      }
+      if constexpr (D == 128) tmem_ld32_at<32>(tO + 32, o);
       tmem_wait_ld();
       tc_fence_before();
-      const float inv_l = 1.0f / l_run;
+      // the row sum is this warp's half plus the other warp's
+      float* lxk = lx + (k & 1) * 2 * kBlockRows;
+      lxk[h * kBlockRows + row] = l_run;
+      mbar_arrive(bar_lx);
+      ok = __all_sync(0xffffffffu, mbar_wait(bar_lx, static_cast<uint32_t>(k) & 1, wc, 13));
+      if (!ok) break;
+      const float inv_l = 1.0f / (l_run + lxk[(h ^ 1) * kBlockRows + row]);
       const int32_t qrow = item.q_row0 + row;
       int64_t out_row = -1;  // destination row, or -1 for no real token
       if constexpr (RASTER) {
@@ -529,9 +549,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         out_row = static_cast<int64_t>(item.bh) * p.L + qrow;
       }
       if (out_row >= 0) {
-        uint4* dst = reinterpret_cast<uint4*>(p.out + out_row * D);
+        uint4* dst = reinterpret_cast<uint4*>(p.out + out_row * D + h * (D / 2));
 #pragma unroll
-        for (int c = 0; c < D / 8; ++c) {
+        for (int c = 0; c < D / 16; ++c) {
           uint4 v4;
           v4.x = pack_bf16x2(__uint_as_float(o[8 * c + 0]) * inv_l, __uint_as_float(o[8 * c + 1]) * inv_l);
           v4.y = pack_bf16x2(__uint_as_float(o[8 * c + 2]) * inv_l, __uint_as_float(o[8 * c + 3]) * inv_l);
@@ -546,7 +566,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == kMmaWarp0) tmem_dealloc(tmem, kTmemCols);
+  if (warp == kPvWarp) tmem_dealloc(tmem, kTmemCols);
 }
 
 // Self-test kernel for the bounded wait: waits on a barrier nobody arrives on.
@@ -623,20 +643,14 @@ cudaError_t launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) return e;
-  // setmaxnreg redistributes the registers a CTA is launched with; the split in
-  // the kernel adds up only if the kernel was compiled to exactly kLaunchRegs.
-  cudaFuncAttributes fa;
-  if ((e = cudaFuncGetAttributes(&fa, kern)) != cudaSuccess) return e;
-  if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
   int dev = 0, sms = 0, per_sm = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
   if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem)) != cudaSuccess) return e;
   if (per_sm < 1) return cudaErrorInvalidConfiguration;
-  // One CTA per SM (two lanes of 128 query rows each; 512 TMEM columns).
+  // One CTA per SM (512 TMEM columns), items strided over the grid.
   int grid = sms;
-  const int pairs = (p.n_items + kLanes - 1) / kLanes;
-  if (grid > pairs) grid = pairs;
+  if (grid > p.n_items) grid = p.n_items;
   if (grid < 1) return cudaSuccess;
   kern<<<grid, kThreads, smem, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
