@@ -21,15 +21,21 @@
 //     TMEM buffers: S of block g+3 is issued as soon as P V of block g has
 //     read P from its buffer, so the scores of the next two blocks are ready
 //     while the softmax works on block g;
-//   * warps 0-7 run the online softmax in fp32, two warps per row: TMEM lane =
-//     query row, warp w and w+4 take key columns 0-63 and 64-127 of the rows of
-//     TMEM lane quadrant w.  Each loads the whole score row for the row max
-//     (no exchange needed), computes p = 2^(s*scale*log2e - m) for its half,
-//     keeps its half of the row sum, and writes its half of P (bf16) over the
-//     first columns of its half of S.  O is rescaled only when the running max
-//     grows by more than 2^8 (O and the row sum always carry the same factor, so
-//     O / l is unchanged); the epilogue adds the two half sums, divides and
-//     writes bf16 rows, each warp half of the head dimension.
+//   * warps 0-7 run the online softmax in fp32: TMEM lane = query row, and the
+//     two warps w and w+4 of TMEM lane quadrant w take the blocks of the CTA's
+//     stream alternately, each handling whole rows (all 128 keys) of its blocks,
+//     so one warp's exponentials overlap the other's loads and hand-offs on the
+//     sub-partition's MUFU unit.  A warp computes p = 2^(s*scale*log2e - m),
+//     keeps its part of the row sum, and writes P (bf16) over the first columns
+//     of each half of S.  The running max m is only a reference point against
+//     overflow: it is the exact row max of the item's first block, and a later
+//     block that exceeds it is still exact as long as p stays finite.  Each
+//     block publishes which rows' reference it set or raised (block row sums
+//     above 2^64 redo the block with their exact max, with O and the row sums
+//     rescaled together, so O / l is unchanged); the other warp reads that
+//     before publishing its next block and redoes rows it computed against the
+//     old reference.  The epilogue adds the two warps' sums, divides and writes
+//     bf16 rows, each warp half of the head dimension.
 //
 // Every barrier that is waited on with a parity can never run two phases ahead
 // of its waiter (the per-buffer S, P and P*V barriers, the Q pair, the ring).
@@ -63,7 +69,7 @@ constexpr int kSWarp = 10;          // issues S = Q K^T
 constexpr int kSBufs = 3;           // score buffers in TMEM
 constexpr int kTmemCols = 512;      // S buffer b at 128 b, O at kOCol
 constexpr int kOCol = 128 * kSBufs;
-constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr float kOverflowSum = 0x1p64f;     // block row sums above this redo the block with its exact max
 constexpr int kDefaultPoly8 = 0;
 
 struct FwdParams {
@@ -93,7 +99,9 @@ struct Smem {
   static constexpr int kQ = 0;                             // Q buffer b at kQ + b * kBlockBytes
   static constexpr int kStage0 = kQBufs * kBlockBytes;     // stage s at kStage0 + s * kBlockBytes
   static constexpr int kLx = kStage0 + kStages * kBlockBytes;  // float [item parity][half][row]
-  static constexpr int kBar = kLx + 2 * 2 * kBlockRows * 4;
+  static constexpr int kOw = kLx + 2 * 2 * kBlockRows * 4;    // uint32 [block parity][quadrant]
+  static constexpr int kOm = kOw + 2 * 4 * 4;                  // float [block parity][row]
+  static constexpr int kBar = kOm + 2 * kBlockRows * 4;
   static constexpr int kQFull = kBar;                      // [Q buffer]
   static constexpr int kQEmpty = kQFull + 16;              // [Q buffer]
   static constexpr int kKvFull = kQEmpty + 16;             // [stage]
@@ -101,8 +109,8 @@ struct Smem {
   static constexpr int kSFull = kKvEmpty + 8 * kStages;    // [S buffer]: S written
   static constexpr int kPFull = kSFull + 8 * kSBufs;       // [S buffer]: P written (8 warps)
   static constexpr int kPvDone = kPFull + 8 * kSBufs;      // [S buffer]: P V of that block completed
-  static constexpr int kSRead = kPvDone + 8 * kSBufs;      // [lane quadrant]: both warps hold S
-  static constexpr int kLxBar = kSRead + 8 * 4;            // [lane quadrant]: half row sums written
+  static constexpr int kOut = kPvDone + 8 * kSBufs;        // [lane quadrant]: outcome of each block published
+  static constexpr int kLxBar = kOut + 8 * 4;              // [lane quadrant]: half row sums written
   static constexpr int kOFull = kLxBar + 8 * 4;
   static constexpr int kDrain = kOFull + 8;
   static constexpr int kDrainS = kDrain + 8;
@@ -181,11 +189,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < kSBufs; ++b) {
       mbar_init(sb + S::kSFull + 8 * b, 1);
-      mbar_init(sb + S::kPFull + 8 * b, 8);    // one arrival per softmax warp
+      mbar_init(sb + S::kPFull + 8 * b, 4);    // one arrival per lane quadrant
       mbar_init(sb + S::kPvDone + 8 * b, 1);
     }
     for (int q = 0; q < 4; ++q) {
-      mbar_init(sb + S::kSRead + 8 * q, 2);    // one arrival per warp of the pair
+      mbar_init(sb + S::kOut + 8 * q, 32);     // every lane of the publishing warp
       mbar_init(sb + S::kLxBar + 8 * q, 64);   // every thread of the pair
     }
     mbar_init(sb + S::kOFull, 1);
@@ -357,209 +365,280 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax + epilogue
-    const int h = warp >> 2;                              // key columns [64 h, 64 h + 64)
+    // Warps w and w+4 share the rows of TMEM lane quadrant w and take the blocks of
+    // the CTA's stream alternately (block g by the warp with h = g mod 2), each
+    // handling whole rows (all 128 keys) of its blocks: while one runs its
+    // exponentials, the other loads, checks and hands over, so the sub-partition's
+    // MUFU unit stays busy.
+    const int h = warp >> 2;
     const int quad = warp & 3;                            // TMEM lane quadrant
     const int row = quad * 32 + lane;                     // TMEM lane = query row in the block
     const uint32_t tlane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
-    const uint32_t tO = tlane + kOCol + h * (D / 2);      // this warp's half of O
-    const uint32_t bar_sread = sb + S::kSRead + 8 * quad, bar_lx = sb + S::kLxBar + 8 * quad;
+    const uint32_t tOrow = tlane + kOCol;                 // the row's O
+    const uint32_t tO = tOrow + h * (D / 2);              // this warp's half of O in the epilogue
+    const uint32_t bar_out = sb + S::kOut + 8 * quad, bar_lx = sb + S::kLxBar + 8 * quad;
+    uint32_t* oword = reinterpret_cast<uint32_t*>(smem + S::kOw);   // [block parity][quadrant]
+    float* omax = reinterpret_cast<float*>(smem + S::kOm);          // [block parity][row]
     float* lx = reinterpret_cast<float*>(smem + S::kLx);
     const float sl2 = p.scale_log2;
-    int32_t g = 0;
+    const bool pad_masks = !MASKED && p.kv_mask_id != nullptr;
     bool ok = true;
-    for (int32_t k = 0; ok; ++k) {
-      const int32_t idx = k * static_cast<int32_t>(gridDim.x) + static_cast<int32_t>(blockIdx.x);
-      if (idx >= p.n_items) break;
-      const WorkItem item = p.items[idx];
-      float m_run = -INFINITY;
-      float l_run = 0.f;   // this warp's half of the row sum
-      // masked path: this row's window box in tile coordinates
-      int32_t ws_t = 0, ws_h = 0, ws_w = 0, we_t = 0, we_h = 0, we_w = 0;
-      if (MASKED) {
-        const int head = item.bh % p.heads;
-        const int32_t et = p.head_win[head * 4 + 0], eh = p.head_win[head * 4 + 1], ew = p.head_win[head * 4 + 2];
-        const int32_t qrow = item.q_row0 + row;
-        const int32_t qt = (qrow < p.L ? qrow : p.L - 1) / p.ntile;
-        const int32_t at = qt / (p.nH * p.nW), ah = (qt / p.nW) % p.nH, aw = qt % p.nW;
-        ws_t = min(max(at - et / 2, 0), p.nT - et); we_t = ws_t + et;
-        ws_h = min(max(ah - eh / 2, 0), p.nH - eh); we_h = ws_h + eh;
-        ws_w = min(max(aw - ew / 2, 0), p.nW - ew); we_w = ws_w + ew;
+    float m_run = -INFINITY;   // reference max of the row (log2 units), shared by the pair
+    float l_run = 0.f;         // this warp's part of the row sum
+    bool have_m = false;       // this warp holds the reference max of the current item
+    int32_t consumed = -1;     // last block whose outcome (published by the other warp) was read
+    int32_t ws_t = 0, ws_h = 0, ws_w = 0, we_t = 0, we_h = 0, we_w = 0;
+    // Outcome of block gg, published by the other warp: the rows whose reference
+    // max it set or raised, with the new value; l follows the same factor as O.
+    auto read_outcome = [&](int32_t gg) -> bool {
+      const bool got = __all_sync(0xffffffffu, mbar_wait(bar_out, static_cast<uint32_t>(gg) & 1, wc, 12));
+      if (!got) return false;
+      const uint32_t word = oword[(gg & 1) * 4 + quad];
+      if ((word >> lane) & 1u) {
+        const float m_new = omax[(gg & 1) * kBlockRows + row];
+        if (m_run != -INFINITY) l_run *= ex2_approx(m_run - m_new);
+        m_run = m_new;
       }
-      for (int j = 0; j < item.kv_len; ++j, ++g) {
+      consumed = gg;
+      return true;
+    };
+    auto publish = [&](int32_t gg, uint32_t word) {
+      if (lane == 0) oword[(gg & 1) * 4 + quad] = word;
+      omax[(gg & 1) * kBlockRows + row] = m_run;
+      mbar_arrive(bar_out);   // every lane: its own omax entry
+    };
+    BlockCursor cur;
+    cur.start(p);
+    while (ok && !cur.done) {
+      const int32_t g = cur.g, j = cur.j;
+      const WorkItem& item = cur.it;
+      if (j == 0) {
+        m_run = -INFINITY;
+        l_run = 0.f;
+        have_m = false;
+        if (MASKED) {
+          const int head = item.bh % p.heads;
+          const int32_t et = p.head_win[head * 4 + 0], eh = p.head_win[head * 4 + 1], ew = p.head_win[head * 4 + 2];
+          const int32_t qrow = item.q_row0 + row;
+          const int32_t qt = (qrow < p.L ? qrow : p.L - 1) / p.ntile;
+          const int32_t at = qt / (p.nH * p.nW), ah = (qt / p.nW) % p.nH, aw = qt % p.nW;
+          ws_t = min(max(at - et / 2, 0), p.nT - et); we_t = ws_t + et;
+          ws_h = min(max(ah - eh / 2, 0), p.nH - eh); we_h = ws_h + eh;
+          ws_w = min(max(aw - ew / 2, 0), p.nW - ew); we_w = ws_w + ew;
+        }
+      }
+      if ((g & 1) == h) {
         const int b = g % kSBufs;
         const uint32_t tS = tlane + 128 * b;
         ok = __all_sync(0xffffffffu, mbar_wait(sb + S::kSFull + 8 * b, (g / kSBufs) & 1, wc, 7));
         if (!ok) break;
         tc_fence_after();
-        // The whole score row in one round trip: this warp's half into r[0, 64),
-        // the other half into r[64, 128) (for the row max only).
-        uint32_t r[128];
-        tmem_ld32_at<0>(tS + 64 * h, r);
-        tmem_ld32_at<32>(tS + 64 * h + 32, r);
-        tmem_ld32_at<64>(tS + 64 * (h ^ 1), r);
-        tmem_ld32_at<96>(tS + 64 * (h ^ 1) + 32, r);
-        tmem_wait_ld();
-        // This warp holds S now: the other warp of the pair may overwrite its half with P.
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar_sread);
-        // r[i] holds key column col(i) of the block
-        auto col = [h](int i) -> int { return i < 64 ? 64 * h + i : 64 * (h ^ 1) + (i - 64); };
-        if (!MASKED && p.kv_mask_id != nullptr) {
-          // padded latent: keys of pad tokens in this block do not exist
-          const int32_t mid = p.kv_mask_id[item.kv_off + j];
-          if (mid >= 0) {
-            const uint4 mw = *reinterpret_cast<const uint4*>(p.kv_masks + 4 * mid);
-            const uint32_t own0 = h ? mw.z : mw.x, own1 = h ? mw.w : mw.y;
-            const uint32_t oth0 = h ? mw.x : mw.z, oth1 = h ? mw.y : mw.w;
-            const uint32_t words[4] = {own0, own1, oth0, oth1};
-#pragma unroll
-            for (int i = 0; i < 128; ++i)
-              if (!((words[i >> 5] >> (i & 31)) & 1u)) r[i] = __float_as_uint(-INFINITY);
+        // Keys [32 c, 32 c + 32) of the block that this row attends, as a bit mask.
+        auto mask_word = [&](int c) -> uint32_t {
+          uint32_t m = 0xffffffffu;
+          if (pad_masks) {
+            // padded latent: keys of pad tokens in this block do not exist
+            const int32_t mid = p.kv_mask_id[item.kv_off + j];
+            if (mid >= 0) m = p.kv_masks[4 * mid + c];
           }
-        }
-        if (MASKED) {
-          const int32_t kv_row = p.kv_rows[item.kv_off + j];
-#pragma unroll
-          for (int i = 0; i < 128; ++i) {
-            const int32_t key = kv_row + col(i);
-            bool in = key < p.L;
-            if (in) {
-              const int32_t kt = key / p.ntile;
-              const int32_t bt = kt / (p.nH * p.nW), bh_ = (kt / p.nW) % p.nH, bw = kt % p.nW;
-              in = bt >= ws_t && bt < we_t && bh_ >= ws_h && bh_ < we_h && bw >= ws_w && bw < we_w;
+          if (MASKED) {
+            const int32_t kv_row = p.kv_rows[item.kv_off + j];
+            m = 0;
+            for (int i = 0; i < 32; ++i) {
+              const int32_t key = kv_row + 32 * c + i;
+              bool in = key < p.L;
+              if (in) {
+                const int32_t kt = key / p.ntile;
+                const int32_t bt = kt / (p.nH * p.nW), bh_ = (kt / p.nW) % p.nH, bw = kt % p.nW;
+                in = bt >= ws_t && bt < we_t && bh_ >= ws_h && bh_ < we_h && bw >= ws_w && bw < we_w;
+              }
+              if (in) m |= 1u << i;
             }
-            if (!in) r[i] = __float_as_uint(-INFINITY);
           }
-        }
-#define SV(i) __uint_as_float(r[i])
-        // Row max: eight independent chains of three-input maxima.
-        float mx8[8];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          float a = max3f(SV(q), SV(q + 8), SV(q + 16));
-#pragma unroll
-          for (int t = 24; t < 120; t += 16) a = max3f(a, SV(q + t), SV(q + t + 8));
-          mx8[q] = fmaxf(a, SV(q + 120));
-        }
-        const float mx = max3f(max3f(mx8[0], mx8[1], mx8[2]), max3f(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
-        const float m_blk = mx * sl2;
-        // The running max moves only when it grows by more than 2^8: p stays <= 256
-        // and O and the row sum always carry the same factor, so O / l is exact.
-        // Both warps of a row see the same scores, so they take the same decision.
-        const bool need = (m_run != -INFINITY) && (m_blk > m_run + kRescaleThreshold);
-        float f = 1.0f;
-        if (m_run == -INFINITY) {
-          m_run = m_blk;  // first contribution to this row: nothing accumulated yet
-        } else if (need) {
-          f = ex2_approx(m_run - m_blk);
-          l_run *= f;
-          m_run = m_blk;
-        }
-        if (__any_sync(0xffffffffu, need)) {
-          // O holds P V up to block g-1, whose product may still be running: wait
-          // for it, then rescale this warp's half of O (tcgen05.ld/st are
-          // warp-collective, so the whole warp takes part).
-          const int pb = (g + kSBufs - 1) % kSBufs;
-          ok = __all_sync(0xffffffffu, mbar_wait(sb + S::kPvDone + 8 * pb, ((g - 1) / kSBufs) & 1, wc, 11));
-          if (!ok) break;
-          tc_fence_after();
-#pragma unroll
-          for (int c = 0; c < D / 64; ++c) {
-            uint32_t o[32];
-            tmem_ld32(tO + c * 32, o);
+          return m;
+        };
+        // Exact row max of S_g, 32 columns at a time (masked keys left out).
+        auto exact_max = [&]() -> float {
+          float mx = -INFINITY;
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            uint32_t v[32];
+            tmem_ld32(tS + 32 * c, v);
             tmem_wait_ld();
+            const uint32_t m = (MASKED || pad_masks) ? mask_word(c) : 0xffffffffu;
+            float a[4];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
-            tmem_st32(tO + c * 32, o);
-          }
-        }
-        const float nm = (m_run == -INFINITY) ? 0.f : -m_run;
-        // p = 2^(s * scale * log2e - m) for this warp's 64 keys: POLY8 of every 8
-        // column pairs on the FMA pipe, the rest on MUFU; x and the row sums use
-        // packed fp32 pairs (one instruction per two columns); four
-        // pair-accumulators break the add chain; P packed to bf16 pairs.
-        const uint64_t sl2x2 = f32x2(sl2, sl2), nmx2 = f32x2(nm, nm);
-        uint64_t ls2[4] = {0, 0, 0, 0};
-        uint32_t pk[32];
+            for (int q = 0; q < 4; ++q) {
+              float x[8];
 #pragma unroll
-        for (int i = 0; i < 64; i += 2) {
-          const uint64_t x2 = fma_f32x2(f32x2(SV(i), SV(i + 1)), sl2x2, nmx2);
-          float p0, p1;
-          float x0, x1;
-          f32x2_split(x2, x0, x1);
-          if (!MASKED && ((i >> 1) & 7) >= 8 - POLY8) {
-            // x >= -125 is kept by the clamp; x <= 8 by the rescale threshold
-            exp2_poly3_pair(f32x2(fmaxf(x0, -125.f), fmaxf(x1, -125.f)), p0, p1);
-          } else {
-            p0 = ex2_approx(x0);
-            p1 = ex2_approx(x1);
+              for (int t = 0; t < 8; ++t)
+                x[t] = ((m >> (q + 4 * t)) & 1u) ? __uint_as_float(v[q + 4 * t]) : -INFINITY;
+              a[q] = max3f(max3f(x[0], x[1], x[2]), max3f(x[3], x[4], x[5]), fmaxf(x[6], x[7]));
+            }
+            mx = max3f(mx, fmaxf(a[0], a[1]), fmaxf(a[2], a[3]));
           }
-          ls2[(i >> 1) & 3] = add_f32x2(ls2[(i >> 1) & 3], f32x2(p0, p1));
-          pk[i >> 1] = pack_bf16x2(p0, p1);
-        }
-#undef SV
-        // P over the first 32 columns of this warp's half of S, once the other warp
-        // of the pair has its copy of S.
-        ok = __all_sync(0xffffffffu, mbar_wait(bar_sread, static_cast<uint32_t>(g) & 1, wc, 12));
-        if (!ok) break;
-        tc_fence_after();
-        tmem_st32_at<0>(tS + 64 * h, pk);
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(sb + S::kPFull + 8 * b);
-        {
+          return mx;
+        };
+        // p = 2^(s * scale * log2e - m) for the whole row, 64 keys at a time: POLY8
+        // of every 8 column pairs on the FMA pipe, the rest on MUFU; x and the row
+        // sums use packed fp32 pairs; P packed to bf16 pairs into pk[32 half + i].
+        // Returns the block's row sum.
+        uint32_t pk[64];
+        auto exps = [&]() -> float {
+          const float nm = (m_run == -INFINITY) ? 0.f : -m_run;
+          const uint64_t sl2x2 = f32x2(sl2, sl2), nmx2 = f32x2(nm, nm);
+          uint64_t ls2[4] = {0, 0, 0, 0};
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            uint32_t r[64];
+            tmem_ld32_at<0>(tS + 64 * hh, r);
+            tmem_ld32_at<32>(tS + 64 * hh + 32, r);
+            tmem_wait_ld();
+            if (MASKED || pad_masks) {
+              const uint32_t m0 = mask_word(2 * hh), m1 = mask_word(2 * hh + 1);
+#pragma unroll
+              for (int i = 0; i < 64; ++i)
+                if (!((((i < 32) ? m0 : m1) >> (i & 31)) & 1u)) r[i] = __float_as_uint(-INFINITY);
+            }
+#pragma unroll
+            for (int i = 0; i < 64; i += 2) {
+              const uint64_t x2 = fma_f32x2(f32x2(__uint_as_float(r[i]), __uint_as_float(r[i + 1])), sl2x2, nmx2);
+              float p0, p1;
+              float x0, x1;
+              f32x2_split(x2, x0, x1);
+              if (!MASKED && ((i >> 1) & 7) >= 8 - POLY8) {
+                // inside [-125, 126] for the cubic; larger x overflow the row sum anyway
+                exp2_poly3_pair(f32x2(fminf(fmaxf(x0, -125.f), 126.f), fminf(fmaxf(x1, -125.f), 126.f)), p0, p1);
+              } else {
+                p0 = ex2_approx(x0);
+                p1 = ex2_approx(x1);
+              }
+              ls2[(i >> 1) & 3] = add_f32x2(ls2[(i >> 1) & 3], f32x2(p0, p1));
+              pk[32 * hh + (i >> 1)] = pack_bf16x2(p0, p1);
+            }
+          }
           float a0, a1, b0, b1, c0, c1, d0, d1;
           f32x2_split(ls2[0], a0, a1);
           f32x2_split(ls2[1], b0, b1);
           f32x2_split(ls2[2], c0, c1);
           f32x2_split(ls2[3], d0, d1);
-          l_run += ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
+          return ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
+        };
+        uint32_t my_word = 0;
+        if (j == 0) {
+          // first block of the item: the exact row max is the reference
+          const float mx = exact_max();
+          m_run = mx * sl2;
+          have_m = true;
+          my_word = 0xffffffffu;
+        } else if (!have_m) {
+          // the other warp took the item's first block: its max is the reference
+          ok = read_outcome(g - 1);
+          if (!ok) break;
+          have_m = true;
         }
-      }
-      if (!ok) break;
-      // epilogue: O / l -> bf16, this warp's half of the head dimension
-      ok = __all_sync(0xffffffffu, mbar_wait(sb + S::kOFull, static_cast<uint32_t>(k) & 1, wc, 8));
-      if (!ok) break;
-      tc_fence_after();
-      uint32_t o[D / 2];
-      tmem_ld32_at<0>(tO, o);
-      if constexpr (D == 128) tmem_ld32_at<32>(tO + 32, o);
-      tmem_wait_ld();
-      tc_fence_before();
-      // the row sum is this warp's half plus the other warp's
-      float* lxk = lx + (k & 1) * 2 * kBlockRows;
-      lxk[h * kBlockRows + row] = l_run;
-      mbar_arrive(bar_lx);
-      ok = __all_sync(0xffffffffu, mbar_wait(bar_lx, static_cast<uint32_t>(k) & 1, wc, 13));
-      if (!ok) break;
-      const float inv_l = 1.0f / (l_run + lxk[(h ^ 1) * kBlockRows + row]);
-      const int32_t qrow = item.q_row0 + row;
-      int64_t out_row = -1;  // destination row, or -1 for no real token
-      if constexpr (RASTER) {
-        const int32_t tile = qrow / p.ntile, local = qrow - tile * p.ntile;
-        const int32_t at = tile / (p.nH * p.nW), ah = (tile / p.nW) % p.nH, aw = tile % p.nW;
-        const int32_t t = at * p.tt + local / (p.th * p.tw);
-        const int32_t hh = ah * p.th + (local / p.tw) % p.th;
-        const int32_t w = aw * p.tw + local % p.tw;
-        if (t < p.T && hh < p.H && w < p.W)
-          out_row = ((static_cast<int64_t>(item.bh) * p.T + t) * p.H + hh) * p.W + w;
-      } else if (qrow < p.L) {
-        out_row = static_cast<int64_t>(item.bh) * p.L + qrow;
-      }
-      if (out_row >= 0) {
-        uint4* dst = reinterpret_cast<uint4*>(p.out + out_row * D + h * (D / 2));
+        float ps = exps();
+        // The reference max is only a guard against overflow: a block that exceeds
+        // it is still exact as long as p stays finite.  Rows whose block sum exceeds
+        // 2^64 (or is not finite), and rows whose reference the other warp raised
+        // in block g-1 (read now, before this block is published), redo the block.
+        uint32_t stale = 0;
+        if (consumed != g - 1 && g > 0) {
+          const float m_before = m_run;
+          ok = read_outcome(g - 1);
+          if (!ok) break;
+          stale = __ballot_sync(0xffffffffu, m_run != m_before);
+        }
+        const uint32_t ovf = (j == 0) ? 0u : __ballot_sync(0xffffffffu, !(ps <= kOverflowSum));
+        if ((ovf | stale) != 0) {
+          float f = 1.0f;
+          if (ovf != 0) {
+            const float mx = exact_max();
+            if ((ovf >> lane) & 1u) {
+              const float m_new = fmaxf(m_run, mx * sl2);
+              f = ex2_approx(m_run - m_new);
+              l_run *= f;
+              m_run = m_new;
+            }
+            // O holds P V up to block g-1, whose product may still be running
+            const int pb = (g + kSBufs - 1) % kSBufs;
+            ok = __all_sync(0xffffffffu, mbar_wait(sb + S::kPvDone + 8 * pb, ((g - 1) / kSBufs) & 1, wc, 11));
+            if (!ok) break;
+            tc_fence_after();
+#pragma unroll 1
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t o[32];
+              tmem_ld32(tOrow + c * 32, o);
+              tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < D / 16; ++c) {
-          uint4 v4;
-          v4.x = pack_bf16x2(__uint_as_float(o[8 * c + 0]) * inv_l, __uint_as_float(o[8 * c + 1]) * inv_l);
-          v4.y = pack_bf16x2(__uint_as_float(o[8 * c + 2]) * inv_l, __uint_as_float(o[8 * c + 3]) * inv_l);
-          v4.z = pack_bf16x2(__uint_as_float(o[8 * c + 4]) * inv_l, __uint_as_float(o[8 * c + 5]) * inv_l);
-          v4.w = pack_bf16x2(__uint_as_float(o[8 * c + 6]) * inv_l, __uint_as_float(o[8 * c + 7]) * inv_l);
-          dst[c] = v4;
+              for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
+              tmem_st32(tOrow + c * 32, o);
+            }
+            my_word = ovf;
+          }
+          ps = exps();
         }
+        publish(g, my_word);
+        // P over the first 32 columns of each half of S_g
+        tmem_st32_at<0>(tS, pk);
+        tmem_st32_at<32>(tS + 64, pk);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(sb + S::kPFull + 8 * b);
+        l_run += ps;
       }
+      if (j + 1 == item.kv_len) {
+        // epilogue: O / l -> bf16, this warp's half of the head dimension.  The
+        // warp that did not take the last block applies its outcome first.
+        const int32_t k = cur.k;
+        if (consumed != g && (g & 1) != h) {
+          ok = read_outcome(g);
+          if (!ok) break;
+        }
+        ok = __all_sync(0xffffffffu, mbar_wait(sb + S::kOFull, static_cast<uint32_t>(k) & 1, wc, 8));
+        if (!ok) break;
+        tc_fence_after();
+        float* lxk = lx + (k & 1) * 2 * kBlockRows;
+        lxk[h * kBlockRows + row] = l_run;
+        mbar_arrive(bar_lx);
+        ok = __all_sync(0xffffffffu, mbar_wait(bar_lx, static_cast<uint32_t>(k) & 1, wc, 13));
+        if (!ok) break;
+        const float inv_l = 1.0f / (l_run + lxk[(h ^ 1) * kBlockRows + row]);
+        const int32_t qrow = item.q_row0 + row;
+        int64_t out_row = -1;  // destination row, or -1 for no real token
+        if constexpr (RASTER) {
+          const int32_t tile = qrow / p.ntile, local = qrow - tile * p.ntile;
+          const int32_t at = tile / (p.nH * p.nW), ah = (tile / p.nW) % p.nH, aw = tile % p.nW;
+          const int32_t t = at * p.tt + local / (p.th * p.tw);
+          const int32_t hh = ah * p.th + (local / p.tw) % p.th;
+          const int32_t w = aw * p.tw + local % p.tw;
+          if (t < p.T && hh < p.H && w < p.W)
+            out_row = ((static_cast<int64_t>(item.bh) * p.T + t) * p.H + hh) * p.W + w;
+        } else if (qrow < p.L) {
+          out_row = static_cast<int64_t>(item.bh) * p.L + qrow;
+        }
+        uint4* dst = reinterpret_cast<uint4*>(p.out + (out_row >= 0 ? out_row : 0) * D + h * (D / 2));
+#pragma unroll 1
+        for (int c32 = 0; c32 < D / 64; ++c32) {
+          uint32_t o[32];
+          tmem_ld32(tO + 32 * c32, o);
+          tmem_wait_ld();
+          if (out_row >= 0) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              uint4 v4;
+              v4.x = pack_bf16x2(__uint_as_float(o[8 * c + 0]) * inv_l, __uint_as_float(o[8 * c + 1]) * inv_l);
+              v4.y = pack_bf16x2(__uint_as_float(o[8 * c + 2]) * inv_l, __uint_as_float(o[8 * c + 3]) * inv_l);
+              v4.z = pack_bf16x2(__uint_as_float(o[8 * c + 4]) * inv_l, __uint_as_float(o[8 * c + 5]) * inv_l);
+              v4.w = pack_bf16x2(__uint_as_float(o[8 * c + 6]) * inv_l, __uint_as_float(o[8 * c + 7]) * inv_l);
+              dst[4 * c32 + c] = v4;
+            }
+          }
+        }
+        tc_fence_before();
+      }
+      cur.next(p);
     }
   }
 
