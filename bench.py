@@ -1,11 +1,12 @@
 """Benchmark of the Sliding Tile Attention forward path on B200.
 
 One step = the whole hot path on one batch of synthetic input: tile reorder of
-q, k and v, tile-windowed attention, reorder of the output back.  With tiles that
-split into 128-row slabs of whole frames (the default workload) that is one
-launch of the fused raster-order kernel; --three-call times the separate
-reorder / tiled attention / unorder kernels instead.  The default workload is the HunyuanVideo-shaped one (latent 30x48x80 = 115200
-tokens, tile (6,8,8), window (3,3,3) tiles, 24 heads, d = 128, bf16).
+q, k and v, tile-windowed attention, reorder of the output back (five launches:
+reorder x3, tiled attention, unorder).  --fused times the one-launch fused
+raster-order kernel as the step instead; the other path is timed beside it and
+reported under `kernels`.  The default workload is the HunyuanVideo-shaped one
+(latent 30x48x80 = 115200 tokens, tile (6,8,8), window (3,3,3) tiles, 24 heads,
+d = 128, bf16).
 
 value = attended FLOPs (4 * d * attended query-key pairs) of all ranks per
 second of step time, device-timed with CUDA events (max over ranks).  Inputs
@@ -34,11 +35,11 @@ if ROOT not in sys.path:
 METRIC = "STA fwd ms & TFLOPS (attended) at 30×48×80, 24 heads, d=128; % of BF16 peak"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-# DRAM bytes (read + write) per launch of the fused raster-order attention kernel on the default
+# DRAM bytes (read + write) per launch of the tiled-order attention kernel on the default
 # workload, from the ncu capture summarised in profiles/sta_fwd_kernel_hunyuan_4heads.md (4-head
 # case, scaled by 6 to 24 heads: traffic is per head).  Valid only for the kernel source it was
 # taken on.
-PROFILED_TRAFFIC = {"sha1": "6a4584f45c0e95d62aebbcf8b8c0db458af052fb", "bytes_per_launch": 6 * (360.189696e6 + 101.390592e6),
+PROFILED_TRAFFIC = {"sha1": "06ba0203e5df56d358c6f7b6a3e71d125a4bdfd9", "bytes_per_launch": 6 * (361.18272e6 + 104.259328e6),
                     "workload": "hunyuan"}
 
 
@@ -227,11 +228,12 @@ def run_ours(args, cfg):
     flops = 4.0 * cfg.d * sta.sta_attended_pairs(cfg.batch, cfg.heads, grid, tile, wins)
     tensor_bytes = q.numel() * q.element_size()
 
-    # One step = the whole hot path on one batch: with a tile that splits into 128-row
-    # slabs of whole frames, one launch of the fused raster-order kernel (tile reorder
-    # in its TMA loads and output addressing); otherwise reorder q, k, v, tiled
-    # attention, unorder (five launches).
-    fused = sta.raster_tile_ok(tile) and not args.three_call
+    # One step = the whole hot path on one batch: reorder q, k, v, tiled attention,
+    # unorder (five launches), or with --fused one launch of the fused raster-order
+    # kernel (tile reorder in its TMA loads and output addressing).
+    if args.fused and not sta.raster_tile_ok(tile):
+        raise SystemExit("--fused needs a tile that splits into 128-row slabs of whole frames")
+    fused = args.fused
     ev = {n: [] for n in ("r0", "r1", "a0", "a1", "u0", "u1")}
 
     def step_three(record: bool, store=ev):
@@ -299,27 +301,46 @@ def run_ours(args, cfg):
     if sta.sta_check_device_status(stream) != sta.STA_OK:
         raise RuntimeError("a kernel gave up on a bounded wait during timing")
 
-    # ---- the three-call path, for its per-kernel figures (not part of `value`)
-    ev3 = {n: [] for n in ("r0", "r1", "a0", "a1", "u0", "u1")}
+    # ---- per-kernel figures of the three-call path (from the timed steps, or from
+    # extra steps when the fused kernel was the step), and the other path's step time
+    # (not part of `value`)
+    hbm = load_peaks().get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"])
+    ev3 = ev if not fused else {n: [] for n in ("r0", "r1", "a0", "a1", "u0", "u1")}
     three = None
-    if args.aux_steps > 0:
+    other = None
+    if fused and args.aux_steps > 0:
         for _ in range(2):
             step_three(False)
         torch.cuda.synchronize()
         for _ in range(args.aux_steps):
             step_three(True, ev3)
         torch.cuda.synchronize()
+    if ev3["r0"]:
         reo_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(ev3["r0"], ev3["r1"])) / 3.0
         uno_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(ev3["u0"], ev3["u1"]))
         att3_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(ev3["a0"], ev3["a1"]))
-        hbm = load_peaks().get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"])
         reo_gbs = 2 * tensor_bytes / (reo_ms * 1e-3) / 1e9
-        three = {"steps": args.aux_steps, "step_ms": 3 * reo_ms + att3_ms + uno_ms,
+        three = {"steps": len(ev3["r0"]), "step_ms": 3 * reo_ms + att3_ms + uno_ms,
                  "tiled_attention_ms": att3_ms, "tiled_attention_tflops": flops / (att3_ms * 1e-3) / 1e12,
                  "reorder_ms_per_tensor": reo_ms, "reorder_gbs": reo_gbs, "reorder_frac_hbm": reo_gbs / hbm,
                  "unorder_ms": uno_ms, "unorder_gbs": 2 * tensor_bytes / (uno_ms * 1e-3) / 1e9}
-        if sta.sta_check_device_status(stream) != sta.STA_OK:
-            raise RuntimeError("a kernel gave up on a bounded wait during the three-call steps")
+    if not fused and args.aux_steps > 0 and sta.raster_tile_ok(tile):
+        evf = {"a0": [], "a1": []}
+        for _ in range(2):
+            sta.sta_attention_fwd_raster(q, k, v, out, grid, tile, wins, scale, stream)
+        torch.cuda.synchronize()
+        for _ in range(args.aux_steps):
+            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            sta.sta_attention_fwd_raster(q, k, v, out, grid, tile, wins, scale, stream)
+            a1.record(stream)
+            evf["a0"].append(a0)
+            evf["a1"].append(a1)
+        torch.cuda.synchronize()
+        f_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(evf["a0"], evf["a1"]))
+        other = {"steps": args.aux_steps, "step_ms": f_ms, "tflops": flops / (f_ms * 1e-3) / 1e12}
+    if sta.sta_check_device_status(stream) != sta.STA_OK:
+        raise RuntimeError("a kernel gave up on a bounded wait during the extra steps")
 
     # ---- end to end through the public API with host buffers
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
@@ -370,7 +391,7 @@ def run_ours(args, cfg):
         "kernels": {"attention_ms": att_ms, "attention_tflops": att_tflops,
                     "path": "fused raster-order kernel, 1 launch per step" if fused else
                             "reorder x3 + tiled attention + unorder, 5 launches per step",
-                    "three_call_path": three},
+                    "three_call_path": three, "fused_path": other},
         "cpu_baseline": cpu,
         "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": 3 * tensor_bytes, "d2h_bytes_per_step": tensor_bytes,
@@ -396,10 +417,10 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=4096)
     ap.add_argument("--ref-rows", type=int, default=512)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--three-call", action="store_true",
-                    help="time the reorder + tiled attention + unorder path as the step")
+    ap.add_argument("--fused", action="store_true",
+                    help="time the one-launch fused raster-order kernel as the step")
     ap.add_argument("--aux-steps", type=int, default=10,
-                    help="extra steps of the three-call path for its per-kernel figures (0: none)")
+                    help="extra steps of the path not timed as the step (0: none)")
     ap.add_argument("--heads", type=int, default=0,
                     help="use only the first N heads of the workload (small profiling cases)")
     args = ap.parse_args()

@@ -224,20 +224,28 @@ def sta_forward(q, k, v, grid, tile, window_per_head, scale: Optional[float] = N
                 stream=None, workspace: Optional[Tuple] = None, fused: Optional[bool] = None):
     """Full STA forward on raster-order [B, heads, L, d] bf16 CUDA tensors.
 
-    With a tile that splits into 128-row slabs of whole frames (``raster_tile_ok``)
-    and ``fused`` not False, one call does everything (``sta_attention_fwd_raster``:
-    tile reorder in the kernel's loads and stores; grids that are not tile multiples
-    are padded).  Otherwise q, k and v are reordered to tiled order, attended and
-    the output reordered back, on ``stream``; ``workspace`` may then hold four
-    preallocated tensors shaped like q (tiled q, k, v and output).  Returns the
-    raster-order output.
+    Two ways, same result:
+
+    * fused: one call does everything (``sta_attention_fwd_raster``: tile reorder in
+      the kernel's loads and stores).  Needs a tile that splits into 128-row slabs
+      of whole frames (``raster_tile_ok``); the only way for grids that are not tile
+      multiples (padding with masking), and the one that needs no scratch memory.
+    * three calls: q, k and v are reordered to tiled order, attended and the output
+      reordered back, on ``stream``; ``workspace`` may hold four preallocated
+      tensors shaped like q (tiled q, k, v and output).  Faster on B200 where both
+      apply (the tiled kernel's K/V loads are plain 3-D boxes of 128 contiguous
+      rows, the fused kernel's are 5-D boxes of whole frames).
+
+    ``fused=None`` takes the fused call only when the grid is not a tile multiple.
+    Returns the raster-order output.
     """
     import torch
     if scale is None:
         scale = 1.0 / float(q.shape[-1]) ** 0.5
     out = torch.empty_like(q)
     if fused is None:
-        fused = raster_tile_ok(tile)
+        multiple = all(int(a) % int(b) == 0 for a, b in zip(grid, tile))
+        fused = not multiple and raster_tile_ok(tile)
     if fused:
         sta_attention_fwd_raster(q, k, v, out, grid, tile, window_per_head, scale, stream)
         return out
