@@ -186,6 +186,23 @@ def run_reference(args, cfg):
 # ---------------------------------------------------------------------------- our arm
 
 
+def max_over_ranks(x: float, device) -> float:
+    """The largest per-rank value over all ranks: a job's time is its slowest rank's.
+    The identity with one process or without an initialised process group."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(world: int, flops_per_rank: float, ms: float) -> float:
+    """Whole-job throughput: every rank processes its own replica of the workload."""
+    return world * flops_per_rank / (ms * 1e-3) / 1e12
+
+
 def config_dict(cfg, args):
     win = sorted(set(cfg.windows))
     return {"workload": f"{cfg.name}: B={cfg.batch}, heads={cfg.heads}, d={cfg.d}, grid={cfg.grid}, "
@@ -290,13 +307,9 @@ def run_ours(args, cfg):
         t_end.record(stream)
         torch.cuda.synchronize()
     barrier()
-    ms_total = t_start.elapsed_time(t_end)
-    if world > 1:
-        tt = torch.tensor([ms_total], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_total = float(tt.item())
+    ms_total = max_over_ranks(t_start.elapsed_time(t_end), dev)
     ms_step = ms_total / args.steps
-    value = world * flops / (ms_step * 1e-3) / 1e12
+    value = job_tflops(world, flops, ms_step)
     att_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(ev["a0"], ev["a1"]))
     if sta.sta_check_device_status(stream) != sta.STA_OK:
         raise RuntimeError("a kernel gave up on a bounded wait during timing")
@@ -358,11 +371,7 @@ def run_ours(args, cfg):
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if world > 1:
-        tt = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dev)
 
     peak_s = peaks.get("bf16_tflops_sustained", PEAKS_FALLBACK["bf16_tflops_sustained"])
     peak_b = peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"])
@@ -393,7 +402,7 @@ def run_ours(args, cfg):
                             "reorder x3 + tiled attention + unorder, 5 launches per step",
                     "three_call_path": three, "fused_path": other},
         "cpu_baseline": cpu,
-        "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS", "ms_per_step": e2e_ms,
+        "e2e": {"value": job_tflops(world, flops, e2e_ms), "unit": "TFLOPS", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": 3 * tensor_bytes, "d2h_bytes_per_step": tensor_bytes,
                 "steps": e2e_steps},
         "clocks": clk.summary(),
