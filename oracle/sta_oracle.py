@@ -1,4 +1,5 @@
-"""Plain CPU oracle for Sliding Tile Attention (STA) forward.
+"""Plain CPU oracle for Sliding Tile Attention (STA): forward, the forward's
+per-row log-sum-exp, and the backward (gradients of q, k and v).
 
 TEST INFRASTRUCTURE ONLY.  Only the tests, the package smoke check and the
 benchmark's CPU-baseline leg may import this module.  The product path (the
@@ -144,6 +145,78 @@ def sta_attention_head(q: np.ndarray, k: np.ndarray, v: np.ndarray, grid, tile, 
         mask = sta_mask(coords[sel], coords, grid, tile, window, pad)
         out[r0:r0 + sel.shape[0]] = masked_softmax_attention(q[sel], k64, v64, mask, scale)
     return out
+
+
+def masked_logsumexp(q: np.ndarray, k: np.ndarray, mask: np.ndarray, scale: float) -> np.ndarray:
+    """Per row, log of the sum over allowed keys of exp(scale * q k^T), natural log,
+    fp64; -inf for a row with no allowed key."""
+    s = scale * (np.asarray(q, dtype=np.float64) @ np.asarray(k, dtype=np.float64).T)
+    s = np.where(mask, s, -np.inf)
+    m = s.max(axis=1)
+    safe = np.where(np.isfinite(m), m, 0.0)
+    return safe + np.log(np.exp(s - safe[:, None]).sum(axis=1))
+
+
+def sta_lse_head(q: np.ndarray, k: np.ndarray, grid, tile, window, scale: float,
+                 rows: Optional[Iterable[int]] = None, pad: bool = False) -> np.ndarray:
+    """Log-sum-exp of each query row's scaled scores over its window's keys (one
+    (batch, head), raster order): the normaliser of the forward's softmax, which
+    a backward pass reuses to rebuild P without a second row max."""
+    L = q.shape[0]
+    coords = raster_coords(grid)
+    rows = np.arange(L) if rows is None else np.asarray(list(rows), dtype=np.int64)
+    row_block = int(min(512, max(16, (1 << 19) // L)))
+    out = np.empty(rows.shape[0], dtype=np.float64)
+    for r0 in range(0, rows.shape[0], row_block):
+        sel = rows[r0:r0 + row_block]
+        out[r0:r0 + sel.shape[0]] = masked_logsumexp(q[sel], k, sta_mask(coords[sel], coords, grid, tile, window, pad),
+                                                     scale)
+    return out
+
+
+def masked_softmax_attention_backward(q: np.ndarray, k: np.ndarray, v: np.ndarray, mask: np.ndarray,
+                                      scale: float, do: np.ndarray):
+    """Gradients of O = softmax(scale * q k^T, masked) v with respect to q, k and v,
+    given dO, by the chain rule written out in fp64:
+
+        P = softmax(S),  dV = P^T dO,  dP = dO V^T,
+        dS_ij = P_ij (dP_ij - D_i) with D_i = sum_j P_ij dP_ij (= dO_i . O_i),
+        dQ = scale dS K,  dK = scale dS^T Q.
+
+    Masked entries have P = 0 and so contribute nothing.  Returns (dq, dk, dv)."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    do = np.asarray(do, dtype=np.float64)
+    _, p = masked_softmax_attention(q, k, v, mask, scale, return_p=True)
+    dv = p.T @ do
+    dp = do @ v.T
+    dd = (p * dp).sum(axis=1, keepdims=True)
+    ds = p * (dp - dd)
+    return scale * (ds @ k), scale * (ds.T @ q), dv
+
+
+def sta_attention_backward_head(q: np.ndarray, k: np.ndarray, v: np.ndarray, do: np.ndarray, grid, tile,
+                                window, scale: float, pad: bool = False):
+    """STA backward of one (batch, head): q, k, v, dO are [L, d] in raster order.
+    Returns fp64 (dq, dk, dv), each [L, d].  Query rows are taken in blocks only to
+    bound memory; dk and dv add up every block's contribution."""
+    L, d = q.shape
+    coords = raster_coords(grid)
+    if coords.shape[0] != L:
+        raise ValueError("q rows do not match the grid")
+    row_block = int(min(512, max(16, (1 << 19) // L)))
+    dq = np.empty((L, d), dtype=np.float64)
+    dk = np.zeros((L, d), dtype=np.float64)
+    dv = np.zeros((L, v.shape[1]), dtype=np.float64)
+    for r0 in range(0, L, row_block):
+        sel = np.arange(r0, min(L, r0 + row_block))
+        mask = sta_mask(coords[sel], coords, grid, tile, window, pad)
+        gq, gk, gv = masked_softmax_attention_backward(q[sel], k, v, mask, scale, do[sel])
+        dq[sel] = gq
+        dk += gk
+        dv += gv
+    return dq, dk, dv
 
 
 def sta_attention(q, k, v, grid, tile, windows, scale: float) -> np.ndarray:

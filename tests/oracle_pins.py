@@ -15,7 +15,10 @@ Sources of the facts pinned here:
     inside each tile), computed with torch's scaled_dot_product_attention in
     fp64;
   * invariants: permutation of tokens, rows of P summing to one, outputs inside
-    the hull of the attended value rows.
+    the hull of the attended value rows;
+  * for the log-sum-exp and the backward: torch.logsumexp and torch autograd of
+    masked scaled_dot_product_attention over the brute-force window, central
+    finite differences through the forward, and the closed-form gradient sums.
 """
 from __future__ import annotations
 
@@ -335,6 +338,87 @@ def pin_padding_is_noop_on_tile_multiples(o):
     assert o.attended_pairs_head(grid, tile, window) == o.attended_pairs_head(grid, tile, window, pad=True)
 
 
+# ----------------------------------------------------------------------------- log-sum-exp and backward
+
+
+def _masked_scores_torch(q, k, grid, tile, window, scale, pad=False):
+    """Scaled scores with the brute-force mask (plain loops) applied, as a torch tensor."""
+    mask = torch.from_numpy(_brute_mask(grid, tile, window, pad))
+    s = scale * (torch.from_numpy(q) @ torch.from_numpy(k).T)
+    return s.masked_fill(~mask, float("-inf")), mask
+
+
+def pin_lse_matches_library(o):
+    """Log-sum-exp over the brute-force window, by torch.logsumexp."""
+    for grid, tile, window, d, pad in [((4, 8, 8), (2, 4, 4), (1, 3, 1), 8, False),
+                                       ((3, 4, 6), (1, 2, 2), (2, 2, 3), 6, False),
+                                       ((5, 7, 9), (2, 4, 4), (3, 3, 3), 4, True)]:
+        L = int(np.prod(grid))
+        q, k, _ = _rand_qkv(L, d, seed=3 * L + d)
+        s, _ = _masked_scores_torch(q, k, grid, tile, window, 0.45, pad)
+        want = torch.logsumexp(s, dim=1).numpy()
+        got = o.sta_lse_head(q, k, grid, tile, window, 0.45, pad=pad)
+        assert np.max(np.abs(got - want)) < 1e-12
+
+
+def _autograd_reference(q, k, v, do, mask, scale):
+    """dq, dk, dv of scaled_dot_product_attention with a boolean mask, by torch autograd."""
+    t = [torch.from_numpy(np.ascontiguousarray(x)).clone().requires_grad_(True) for x in (q, k, v)]
+    out = torch.nn.functional.scaled_dot_product_attention(*[x[None, None] for x in t], attn_mask=mask[None, None],
+                                                           scale=scale)[0, 0]
+    out.backward(torch.from_numpy(np.ascontiguousarray(do)))
+    return [x.grad.numpy() for x in t]
+
+
+def pin_backward_equals_autograd(o):
+    """Dense, per-tile and padded windows against torch autograd of masked SDPA."""
+    for grid, tile, window, d, pad in [((4, 8, 8), (2, 4, 4), (3, 3, 3), 8, False),   # window = grid: dense
+                                       ((4, 8, 8), (2, 4, 4), (1, 1, 1), 8, False),   # per tile
+                                       ((3, 6, 8), (1, 2, 4), (1, 3, 1), 6, False),
+                                       ((5, 7, 9), (2, 4, 4), (1, 3, 3), 4, True)]:
+        L = int(np.prod(grid))
+        q, k, v = _rand_qkv(L, d, seed=7 * L + d)
+        do = _rand_qkv(L, d, seed=L)[0]
+        mask = torch.from_numpy(_brute_mask(grid, tile, window, pad))
+        want = _autograd_reference(q, k, v, do, mask, 0.6)
+        got = o.sta_attention_backward_head(q, k, v, do, grid, tile, window, 0.6, pad=pad)
+        for g, w in zip(got, want):
+            assert np.max(np.abs(g - w)) < 1e-11
+
+
+def pin_backward_finite_differences(o):
+    """Central differences of sum(O * dO) through the (separately pinned) forward."""
+    grid, tile, window, d, scale = (2, 4, 4), (1, 2, 2), (1, 3, 1), 4, 0.7
+    L = 32
+    q, k, v = _rand_qkv(L, d, seed=11)
+    do = _rand_qkv(L, d, seed=12)[0]
+    grads = o.sta_attention_backward_head(q, k, v, do, grid, tile, window, scale)
+    rng = np.random.default_rng(13)
+    h = 1e-6
+    for which in range(3):
+        for _ in range(8):
+            i, j = int(rng.integers(L)), int(rng.integers(d))
+            args = [q.copy(), k.copy(), v.copy()]
+            args[which][i, j] += h
+            fp = np.sum(o.sta_attention_head(*args, grid, tile, window, scale) * do)
+            args[which][i, j] -= 2 * h
+            fm = np.sum(o.sta_attention_head(*args, grid, tile, window, scale) * do)
+            fd = (fp - fm) / (2 * h)
+            assert abs(fd - grads[which][i, j]) < 1e-6 * max(1.0, abs(fd)), (which, i, j, fd, grads[which][i, j])
+
+
+def pin_backward_closed_forms(o):
+    """Rows of P sum to one, so the value gradients sum to the output gradients;
+    rows of dS sum to zero, so the key gradients sum to zero."""
+    grid, tile, window, d = (3, 8, 8), (1, 4, 4), (1, 1, 3), 8
+    L = int(np.prod(grid))
+    q, k, v = _rand_qkv(L, d, seed=21)
+    do = _rand_qkv(L, d, seed=22)[0]
+    dq, dk, dv = o.sta_attention_backward_head(q, k, v, do, grid, tile, window, 0.3)
+    assert np.max(np.abs(dv.sum(axis=0) - do.sum(axis=0))) < 1e-10
+    assert np.max(np.abs(dk.sum(axis=0))) < 1e-10
+
+
 ALL_PINS = [
     pin_index_map_golden,
     pin_index_map_properties,
@@ -352,4 +436,8 @@ ALL_PINS = [
     pin_padding_brute_force,
     pin_padding_equals_explicit_padded_grid,
     pin_padding_is_noop_on_tile_multiples,
+    pin_lse_matches_library,
+    pin_backward_equals_autograd,
+    pin_backward_finite_differences,
+    pin_backward_closed_forms,
 ]

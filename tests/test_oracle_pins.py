@@ -93,7 +93,32 @@ def _mut_pad_floor(grid, tile, pad=False):
     return _orig_tile_grid(grid, tile, pad)
 
 
+def _mut_bwd_no_d_term(q, k, v, mask, scale, do):
+    _, p = _orig_msa(q, k, v, mask, scale, return_p=True)
+    dp = np.asarray(do, float) @ np.asarray(v, float).T
+    ds = p * dp
+    return scale * (ds @ np.asarray(k, float)), scale * (ds.T @ np.asarray(q, float)), p.T @ np.asarray(do, float)
+
+
+def _mut_bwd_dq_unscaled(q, k, v, mask, scale, do):
+    dq, dk, dv = _orig_bwd(q, k, v, mask, scale, do)
+    return dq / scale, dk, dv
+
+
+def _mut_bwd_dv_unnormalised(q, k, v, mask, scale, do):
+    dq, dk, _ = _orig_bwd(q, k, v, mask, scale, do)
+    s = scale * (np.asarray(q, float) @ np.asarray(k, float).T)
+    e = np.exp(np.where(mask, s, -np.inf) - s.max(axis=1, keepdims=True))
+    return dq, dk, e.T @ np.asarray(do, float)
+
+
+def _mut_lse_base2(q, k, mask, scale):
+    return _orig_lse(q, k, mask, scale) / np.log(2.0)
+
+
 _orig_msa = O.masked_softmax_attention
+_orig_bwd = O.masked_softmax_attention_backward
+_orig_lse = O.masked_logsumexp
 _orig_mask = O.sta_mask
 _orig_tile_grid = O.tile_grid
 
@@ -110,6 +135,10 @@ MUTANTS = {
     "mask_transposed": ("sta_mask", _mut_mask_transposed),
     "token_granular_window": ("sta_mask", _mut_mask_token_granular),
     "padded_tile_grid_rounded_down": ("tile_grid", _mut_pad_floor),
+    "backward_without_row_term": ("masked_softmax_attention_backward", _mut_bwd_no_d_term),
+    "backward_dq_unscaled": ("masked_softmax_attention_backward", _mut_bwd_dq_unscaled),
+    "backward_dv_unnormalised": ("masked_softmax_attention_backward", _mut_bwd_dv_unnormalised),
+    "logsumexp_in_base_2": ("masked_logsumexp", _mut_lse_base2),
 }
 
 
