@@ -355,6 +355,39 @@ def run_ours(args, cfg):
     if sta.sta_check_device_status(stream) != sta.STA_OK:
         raise RuntimeError("a kernel gave up on a bounded wait during the extra steps")
 
+    # ---- the backward pass (not part of `value`): forward with log-sum-exp on the
+    # tiled tensors, then sta_attention_bwd; algorithmic work 10 d FLOPs per pair
+    # (S, dP, dV, dQ, dK)
+    backward = None
+    ntile = tile[0] * tile[1] * tile[2]
+    if args.backward_steps > 0 and ntile % 128 == 0:
+        lse = torch.empty(cfg.batch, cfg.heads, cfg.L, device=dev, dtype=torch.float32)
+        for src, dst in ((q, qt), (k, kt), (v, vt)):
+            sta.sta_tile_reorder(src, dst, grid, tile, stream)
+        sta.sta_attention_fwd_lse(qt, kt, vt, ot, lse, grid, tile, wins, scale, stream)
+        dot = torch.empty_like(q)
+        sta.sta_tile_reorder(q, dot, grid, tile, stream)   # any bf16 tensor serves as dO
+        grads = [torch.empty_like(q) for _ in range(3)]
+        for _ in range(2):
+            sta.sta_attention_bwd(qt, kt, vt, ot, dot, lse, *grads, grid, tile, wins, scale, stream)
+        torch.cuda.synchronize()
+        b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        b0.record(stream)
+        for _ in range(args.backward_steps):
+            sta.sta_attention_bwd(qt, kt, vt, ot, dot, lse, *grads, grid, tile, wins, scale, stream)
+        b1.record(stream)
+        torch.cuda.synchronize()
+        if sta.sta_check_device_status(stream) != sta.STA_OK:
+            raise RuntimeError("a kernel gave up on a bounded wait during the backward steps")
+        bwd_ms = b0.elapsed_time(b1) / args.backward_steps
+        bwd_tf = 2.5 * flops / (bwd_ms * 1e-3) / 1e12
+        backward = {"steps": args.backward_steps, "ms": bwd_ms, "tflops": bwd_tf,
+                    "frac_of_sustained": bwd_tf / peaks.get("bf16_tflops_sustained", PEAKS_FALLBACK["bf16_tflops_sustained"]),
+                    "launches_per_step": 3,
+                    "work": "10 d FLOPs per attended pair (S, dP, dV, dQ, dK); the kernels recompute S and dP "
+                            "in both the dQ and the dK/dV pass (14 d executed)"}
+        del lse, dot, grads
+
     # ---- end to end through the public API with host buffers
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
     barrier()
@@ -400,7 +433,7 @@ def run_ours(args, cfg):
         "kernels": {"attention_ms": att_ms, "attention_tflops": att_tflops,
                     "path": "fused raster-order kernel, 1 launch per step" if fused else
                             "reorder x3 + tiled attention + unorder, 5 launches per step",
-                    "three_call_path": three, "fused_path": other},
+                    "three_call_path": three, "fused_path": other, "backward": backward},
         "cpu_baseline": cpu,
         "e2e": {"value": job_tflops(world, flops, e2e_ms), "unit": "TFLOPS", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": 3 * tensor_bytes, "d2h_bytes_per_step": tensor_bytes,
@@ -430,6 +463,8 @@ def main():
                     help="time the one-launch fused raster-order kernel as the step")
     ap.add_argument("--aux-steps", type=int, default=10,
                     help="extra steps of the path not timed as the step (0: none)")
+    ap.add_argument("--backward-steps", type=int, default=5,
+                    help="timed steps of the backward pass, reported beside the forward (0: none)")
     ap.add_argument("--heads", type=int, default=0,
                     help="use only the first N heads of the workload (small profiling cases)")
     args = ap.parse_args()

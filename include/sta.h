@@ -117,6 +117,46 @@ sta_status sta_attention_fwd(const void* q, const void* k, const void* v, void* 
                              void* stream);
 
 /*
+ * sta_attention_fwd that also returns each query row's log-sum-exp: the
+ * normaliser of the row's softmax, lse[i] = log(sum_j exp(scale * q_i . k_j)) over
+ * the keys j of the row's window (natural log), which a backward pass uses to
+ * rebuild the probabilities without a second row maximum.
+ *   lse: device fp32 [batch, heads, L], tiled order like q (row n of the tiled
+ *   tensors), 4-byte aligned, not overlapping q, k, v or out.
+ * Everything else as sta_attention_fwd.
+ * Errors: those of sta_attention_fwd; NULL also for a null lse, ALIGN for an
+ * unaligned lse, ALIAS for an lse overlapping another tensor.
+ */
+sta_status sta_attention_fwd_lse(const void* q, const void* k, const void* v, void* out, float* lse,
+                                 int32_t batch, int32_t heads, int32_t d, sta_dim3 grid,
+                                 sta_dim3 tile, const sta_dim3* window_per_head, float scale,
+                                 void* stream);
+
+/*
+ * STA backward pass ("Fast Video Generation with Sliding Tile Attention": the
+ * gradients of the tile-windowed attention of sta_attention_fwd, for the
+ * fine-tuning the paper describes).  With P = softmax(scale q k^T) over each row's
+ * window, rebuilt from lse:
+ *   dv = P^T dout,  ds = P (dout v^T - D) with D_i = dout_i . out_i,
+ *   dq = scale ds k,  dk = scale ds^T q.
+ *   q, k, v, out, dout: device bf16 [batch, heads, L, d], tiled order, as passed to
+ *   and returned by sta_attention_fwd_lse; lse: its fp32 [batch, heads, L] output.
+ *   dq, dk, dv: device bf16 [batch, heads, L, d], tiled order, written.
+ *   All 16-byte aligned; the outputs overlap no input and no other output.
+ * Arithmetic: bf16 operands, fp32 tensor-core accumulation, P and ds rounded to
+ * bf16 for the products that take them, bf16 results.
+ * The tile must hold a multiple of 128 tokens (for example (6,8,8) or (1,8,16)).
+ * The library keeps one fp32 per query row of scratch (grown on demand, freed by
+ * sta_shutdown), so the first call of a larger size synchronises the device.
+ * Errors: NULL, ALIGN, ALIAS, SHAPE (also: tile not a multiple of 128 tokens),
+ * WINDOW, HEADDIM, ARG, ARCH, CUDA.
+ */
+sta_status sta_attention_bwd(const void* q, const void* k, const void* v, const void* out, const void* dout,
+                             const float* lse, void* dq, void* dk, void* dv, int32_t batch, int32_t heads,
+                             int32_t d, sta_dim3 grid, sta_dim3 tile, const sta_dim3* window_per_head,
+                             float scale, void* stream);
+
+/*
  * STA forward on raster-order tensors, with the tile reorder fused into the
  * kernel's loads and stores, and padding with masking ("Fast Video Generation with
  * Sliding Tile Attention", review reply on input resolution): the grid need not be

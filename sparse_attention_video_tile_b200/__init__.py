@@ -60,6 +60,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "sta_tile_unorder": (ctypes.c_int, [P, P, I64, I32, D3, D3, P]),
         "sta_attention_fwd": (ctypes.c_int, [P, P, P, P, I32, I32, I32, D3, D3, ctypes.POINTER(D3), F, P]),
         "sta_attention_fwd_raster": (ctypes.c_int, [P, P, P, P, I32, I32, I32, D3, D3, ctypes.POINTER(D3), F, P]),
+        "sta_attention_fwd_lse": (ctypes.c_int, [P, P, P, P, P, I32, I32, I32, D3, D3, ctypes.POINTER(D3), F, P]),
+        "sta_attention_bwd": (ctypes.c_int, [P, P, P, P, P, P, P, P, P, I32, I32, I32, D3, D3, ctypes.POINTER(D3), F, P]),
         "sta_check_device_status": (ctypes.c_int, [P]),
         "sta_selftest_bounded_wait": (ctypes.c_int, [U64, P]),
         "sta_shutdown": (None, []),
@@ -173,6 +175,53 @@ def sta_attention_fwd(q, k, v, out, grid, tile, window_per_head, scale: float, s
                                           _tensor_ptr(out, "out"), B, Hn, d, _d3(grid), _d3(tile),
                                           _windows(window_per_head), float(scale), _stream(stream))
     _check(st, "sta_attention_fwd")
+
+
+def sta_attention_fwd_lse(q, k, v, out, lse, grid, tile, window_per_head, scale: float, stream=None) -> None:
+    """sta_attention_fwd that also writes each row's log-sum-exp into ``lse``, an fp32
+    CUDA tensor [B, heads, L] (tiled order)."""
+    import torch
+    if q.dim() != 4:
+        raise ValueError("q must be [batch, heads, L, d]")
+    B, Hn, L, d = (int(x) for x in q.shape)
+    for name, t in (("k", k), ("v", v), ("out", out)):
+        if tuple(t.shape) != tuple(q.shape):
+            raise ValueError(f"{name} shape {tuple(t.shape)} differs from q {tuple(q.shape)}")
+    if not isinstance(lse, torch.Tensor) or lse.dtype != torch.float32 or not lse.is_cuda or not lse.is_contiguous():
+        raise TypeError("lse must be a contiguous float32 CUDA tensor")
+    if tuple(lse.shape) != (B, Hn, L):
+        raise ValueError(f"lse must be [batch, heads, L] = {(B, Hn, L)}")
+    if len(window_per_head) != Hn:
+        raise ValueError("one window per head is required")
+    st = load_library().sta_attention_fwd_lse(_tensor_ptr(q, "q"), _tensor_ptr(k, "k"), _tensor_ptr(v, "v"),
+                                              _tensor_ptr(out, "out"), lse.data_ptr(), B, Hn, d, _d3(grid),
+                                              _d3(tile), _windows(window_per_head), float(scale), _stream(stream))
+    _check(st, "sta_attention_fwd_lse")
+
+
+def sta_attention_bwd(q, k, v, out, dout, lse, dq, dk, dv, grid, tile, window_per_head, scale: float,
+                      stream=None) -> None:
+    """STA backward on tiled-order [B, heads, L, d] bf16 CUDA tensors: writes dq, dk,
+    dv from the forward's inputs, output and log-sum-exp (fp32 [B, heads, L]) and
+    the output gradient dout."""
+    import torch
+    if q.dim() != 4:
+        raise ValueError("q must be [batch, heads, L, d]")
+    B, Hn, L, d = (int(x) for x in q.shape)
+    for name, t in (("k", k), ("v", v), ("out", out), ("dout", dout), ("dq", dq), ("dk", dk), ("dv", dv)):
+        if tuple(t.shape) != tuple(q.shape):
+            raise ValueError(f"{name} shape {tuple(t.shape)} differs from q {tuple(q.shape)}")
+    if not isinstance(lse, torch.Tensor) or lse.dtype != torch.float32 or not lse.is_cuda or not lse.is_contiguous():
+        raise TypeError("lse must be a contiguous float32 CUDA tensor")
+    if tuple(lse.shape) != (B, Hn, L):
+        raise ValueError(f"lse must be [batch, heads, L] = {(B, Hn, L)}")
+    if len(window_per_head) != Hn:
+        raise ValueError("one window per head is required")
+    ptrs = [_tensor_ptr(t, n) for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout"))]
+    outs = [_tensor_ptr(t, n) for t, n in ((dq, "dq"), (dk, "dk"), (dv, "dv"))]
+    st = load_library().sta_attention_bwd(*ptrs, lse.data_ptr(), *outs, B, Hn, d, _d3(grid), _d3(tile),
+                                          _windows(window_per_head), float(scale), _stream(stream))
+    _check(st, "sta_attention_bwd")
 
 
 def sta_attention_fwd_raster(q, k, v, out, grid, tile, window_per_head, scale: float, stream=None) -> None:

@@ -19,7 +19,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libsta.so")
 BUILD_DIR = os.path.join(ROOT, "_build")
 
-SOURCES = ["api.cu", "attention.cu", "noalloc.cu", "reorder.cu", "schedule.cpp"]
+SOURCES = ["api.cu", "attention.cu", "backward.cu", "noalloc.cu", "reorder.cu", "schedule.cpp"]
 HEADERS = ["internal.h", "ptx.cuh"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

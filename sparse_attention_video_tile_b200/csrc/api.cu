@@ -57,12 +57,15 @@ struct CachedSchedule {
   uint32_t* d_kv_masks = nullptr;
 };
 
-// (raster, batch, heads, T, H, W, tt, th, tw, windows)
+// (kind, batch, heads, T, H, W, tt, th, tw, windows); kind 0 = tiled order, 1 = raster
+// order (padded), 2 = transposed (key blocks with their query blocks, for the backward)
 using ScheduleKey = std::tuple<int32_t, int32_t, int32_t, int32_t, int32_t, int32_t, int32_t, int32_t, int32_t,
                                std::vector<int32_t>>;
 
 struct DeviceState {
   int32_t* d_err = nullptr;  // bounded-wait status word
+  float* d_dvec = nullptr;   // backward scratch: one float per query row
+  size_t dvec_rows = 0;
   std::list<std::pair<ScheduleKey, std::unique_ptr<CachedSchedule>>> schedules;  // most recent first
 };
 
@@ -106,14 +109,14 @@ cudaError_t upload(T** dst, const std::vector<T>& v) {
 
 // Caller holds g_mu.
 sta_status get_schedule(DeviceState* st, const Geometry& g, int32_t batch, int32_t heads,
-                        const sta_dim3* windows, bool raster, CachedSchedule** out) {
+                        const sta_dim3* windows, int kind, CachedSchedule** out) {
   std::vector<int32_t> wv(static_cast<size_t>(heads) * 3);
   for (int32_t h = 0; h < heads; ++h) {
     wv[h * 3 + 0] = windows[h].t;
     wv[h * 3 + 1] = windows[h].h;
     wv[h * 3 + 2] = windows[h].w;
   }
-  ScheduleKey key{raster ? 1 : 0, batch, heads, g.T, g.H, g.W, g.tt, g.th, g.tw, std::move(wv)};
+  ScheduleKey key{kind, batch, heads, g.T, g.H, g.W, g.tt, g.th, g.tw, std::move(wv)};
   for (auto it = st->schedules.begin(); it != st->schedules.end(); ++it) {
     if (it->first == key) {
       st->schedules.splice(st->schedules.begin(), st->schedules, it);
@@ -122,8 +125,10 @@ sta_status get_schedule(DeviceState* st, const Geometry& g, int32_t batch, int32
     }
   }
   auto cs = std::make_unique<CachedSchedule>();
-  if (raster)
+  if (kind == 1)
     build_schedule_raster(g, batch, heads, windows, &cs->host);
+  else if (kind == 2)
+    build_schedule_transposed(g, batch, heads, windows, &cs->host);
   else
     build_schedule(g, batch, heads, windows, &cs->host);
   for (const WorkItem& w : cs->host.items)
@@ -238,11 +243,14 @@ sta_status sta_tile_unorder(const void* src, void* dst, int64_t batch_heads, int
   return e == cudaSuccess ? STA_OK : cuda_fail(e);
 }
 
-sta_status sta_attention_fwd(const void* q, const void* k, const void* v, void* out, int32_t batch,
-                             int32_t heads, int32_t d, sta_dim3 grid, sta_dim3 tile,
-                             const sta_dim3* window_per_head, float scale, void* stream) {
+namespace {
+// sta_attention_fwd and sta_attention_fwd_lse: validation, schedule, launch.
+sta_status attention_fwd_impl(const void* q, const void* k, const void* v, void* out, float* lse, int32_t batch,
+                              int32_t heads, int32_t d, sta_dim3 grid, sta_dim3 tile,
+                              const sta_dim3* window_per_head, float scale, void* stream) {
   if (!q || !k || !v || !out || !window_per_head) return STA_ERR_NULL;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return STA_ERR_ALIGN;
+  if (lse && reinterpret_cast<uintptr_t>(lse) % 4 != 0) return STA_ERR_ALIGN;
   if (d != 64 && d != 128) return STA_ERR_HEADDIM;
   Geometry g;
   sta_status s = make_geometry(grid, tile, &g);
@@ -253,6 +261,15 @@ sta_status sta_attention_fwd(const void* q, const void* k, const void* v, void* 
     if (window_per_head[h].t < 1 || window_per_head[h].h < 1 || window_per_head[h].w < 1) return STA_ERR_WINDOW;
   const int64_t bytes = static_cast<int64_t>(batch) * heads * g.L * d * 2;
   if (overlaps(out, q, bytes) || overlaps(out, k, bytes) || overlaps(out, v, bytes)) return STA_ERR_ALIAS;
+  if (lse) {
+    const int64_t lbytes = static_cast<int64_t>(batch) * heads * g.L * 4;
+    auto hit = [&](const void* t) {
+      const char* a = static_cast<const char*>(t);
+      const char* b = reinterpret_cast<const char*>(lse);
+      return a < b + lbytes && b < a + bytes;
+    };
+    if (hit(q) || hit(k) || hit(v) || hit(out)) return STA_ERR_ALIAS;
+  }
   int dev = 0;
   if ((s = check_device(&dev)) != STA_OK) return s;
 
@@ -260,11 +277,86 @@ sta_status sta_attention_fwd(const void* q, const void* k, const void* v, void* 
   DeviceState* st = nullptr;
   if ((s = device_state(dev, &st)) != STA_OK) return s;
   CachedSchedule* cs = nullptr;
-  if ((s = get_schedule(st, g, batch, heads, window_per_head, false, &cs)) != STA_OK) return s;
+  if ((s = get_schedule(st, g, batch, heads, window_per_head, 0, &cs)) != STA_OK) return s;
   DeviceSchedule ds{cs->d_items, cs->d_kv_rows, cs->d_head_win, static_cast<int32_t>(cs->host.items.size()),
                     cs->host.masked};
   cudaError_t e = launch_attention(q, k, v, out, batch, heads, d, g, ds, scale, st->d_err, kWaitLimitNs,
-                                   static_cast<cudaStream_t>(stream));
+                                   static_cast<cudaStream_t>(stream), lse);
+  return e == cudaSuccess ? STA_OK : cuda_fail(e);
+}
+}  // namespace
+
+sta_status sta_attention_fwd(const void* q, const void* k, const void* v, void* out, int32_t batch,
+                             int32_t heads, int32_t d, sta_dim3 grid, sta_dim3 tile,
+                             const sta_dim3* window_per_head, float scale, void* stream) {
+  return attention_fwd_impl(q, k, v, out, nullptr, batch, heads, d, grid, tile, window_per_head, scale, stream);
+}
+
+sta_status sta_attention_fwd_lse(const void* q, const void* k, const void* v, void* out, float* lse,
+                                 int32_t batch, int32_t heads, int32_t d, sta_dim3 grid, sta_dim3 tile,
+                                 const sta_dim3* window_per_head, float scale, void* stream) {
+  if (!lse) return STA_ERR_NULL;
+  return attention_fwd_impl(q, k, v, out, lse, batch, heads, d, grid, tile, window_per_head, scale, stream);
+}
+
+sta_status sta_attention_bwd(const void* q, const void* k, const void* v, const void* out, const void* dout,
+                             const float* lse, void* dq, void* dk, void* dv, int32_t batch, int32_t heads,
+                             int32_t d, sta_dim3 grid, sta_dim3 tile, const sta_dim3* window_per_head, float scale,
+                             void* stream) {
+  if (!q || !k || !v || !out || !dout || !lse || !dq || !dk || !dv || !window_per_head) return STA_ERR_NULL;
+  const void* bf[8] = {q, k, v, out, dout, dq, dk, dv};
+  for (const void* t : bf)
+    if (!aligned16(t)) return STA_ERR_ALIGN;
+  if (!aligned16(lse)) return STA_ERR_ALIGN;
+  if (d != 64 && d != 128) return STA_ERR_HEADDIM;
+  Geometry g;
+  sta_status s = make_geometry(grid, tile, &g);
+  if (s != STA_OK) return s;
+  if (g.ntile % kBlockRows != 0) return STA_ERR_SHAPE;
+  if (batch < 1 || heads < 1 || static_cast<int64_t>(batch) * heads > (int64_t(1) << 24)) return STA_ERR_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return STA_ERR_ARG;
+  for (int32_t h = 0; h < heads; ++h)
+    if (window_per_head[h].t < 1 || window_per_head[h].h < 1 || window_per_head[h].w < 1) return STA_ERR_WINDOW;
+  const int64_t rows = static_cast<int64_t>(batch) * heads * g.L;
+  const int64_t bytes = rows * d * 2;
+  // each output overlaps no other tensor
+  const void* outs[3] = {dq, dk, dv};
+  for (int i = 0; i < 3; ++i) {
+    for (int j = 0; j < 5; ++j)
+      if (overlaps(outs[i], bf[j], bytes)) return STA_ERR_ALIAS;
+    for (int j = i + 1; j < 3; ++j)
+      if (overlaps(outs[i], outs[j], bytes)) return STA_ERR_ALIAS;
+    const char* a = static_cast<const char*>(outs[i]);
+    const char* l = reinterpret_cast<const char*>(lse);
+    if (a < l + rows * 4 && l < a + bytes) return STA_ERR_ALIAS;
+  }
+  int dev = 0;
+  if ((s = check_device(&dev)) != STA_OK) return s;
+
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState* st = nullptr;
+  if ((s = device_state(dev, &st)) != STA_OK) return s;
+  if (st->dvec_rows < static_cast<size_t>(rows)) {
+    // grows only; kept for later calls (stream-ordered use, so the old buffer is
+    // freed after synchronising)
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (st->d_dvec) cudaFree(st->d_dvec);
+    st->d_dvec = nullptr;
+    st->dvec_rows = 0;
+    if ((e = cudaMalloc(&st->d_dvec, static_cast<size_t>(rows) * sizeof(float))) != cudaSuccess) return cuda_fail(e);
+    st->dvec_rows = static_cast<size_t>(rows);
+  }
+  CachedSchedule* fw = nullptr;
+  if ((s = get_schedule(st, g, batch, heads, window_per_head, 0, &fw)) != STA_OK) return s;
+  CachedSchedule* tr = nullptr;
+  if ((s = get_schedule(st, g, batch, heads, window_per_head, 2, &tr)) != STA_OK) return s;
+  // a new schedule may have evicted the other from the cache: look the forward one up again
+  if ((s = get_schedule(st, g, batch, heads, window_per_head, 0, &fw)) != STA_OK) return s;
+  DeviceSchedule dfw{fw->d_items, fw->d_kv_rows, fw->d_head_win, static_cast<int32_t>(fw->host.items.size()), false};
+  DeviceSchedule dtr{tr->d_items, tr->d_kv_rows, tr->d_head_win, static_cast<int32_t>(tr->host.items.size()), false};
+  cudaError_t e = launch_backward(q, k, v, out, dout, lse, st->d_dvec, dq, dk, dv, batch, heads, d, g, dfw, dtr,
+                                  scale, st->d_err, kWaitLimitNs, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? STA_OK : cuda_fail(e);
 }
 
@@ -291,7 +383,7 @@ sta_status sta_attention_fwd_raster(const void* q, const void* k, const void* v,
   DeviceState* st = nullptr;
   if ((s = device_state(dev, &st)) != STA_OK) return s;
   CachedSchedule* cs = nullptr;
-  if ((s = get_schedule(st, g, batch, heads, window_per_head, true, &cs)) != STA_OK) return s;
+  if ((s = get_schedule(st, g, batch, heads, window_per_head, 1, &cs)) != STA_OK) return s;
   DeviceSchedule ds{cs->d_items, cs->d_kv_rows, cs->d_head_win, static_cast<int32_t>(cs->host.items.size()), false,
                     cs->d_kv_mask_id, cs->d_kv_masks};
   cudaError_t e = launch_attention_raster(q, k, v, out, batch, heads, d, g, ds, scale, st->d_err, kWaitLimitNs,
@@ -345,6 +437,9 @@ void sta_shutdown(void) {
     kv.second.schedules.clear();
     if (kv.second.d_err) cudaFree(kv.second.d_err);
     kv.second.d_err = nullptr;
+    if (kv.second.d_dvec) cudaFree(kv.second.d_dvec);
+    kv.second.d_dvec = nullptr;
+    kv.second.dvec_rows = 0;
   }
   g_devices.clear();
   cudaSetDevice(cur);

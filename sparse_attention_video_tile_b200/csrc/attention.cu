@@ -89,6 +89,7 @@ struct FwdParams {
   float scale_log2;          // scale * log2(e)
   int32_t* err;
   uint64_t limit_ns;
+  float* lse;                // per-row log-sum-exp (natural log), same row indexing as out, or null
 };
 
 template <int D>
@@ -604,7 +605,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(bar_lx);
         ok = __all_sync(0xffffffffu, mbar_wait(bar_lx, static_cast<uint32_t>(k) & 1, wc, 13));
         if (!ok) break;
-        const float inv_l = 1.0f / (l_run + lxk[(h ^ 1) * kBlockRows + row]);
+        const float l_tot = l_run + lxk[(h ^ 1) * kBlockRows + row];
+        const float inv_l = 1.0f / l_tot;
         const int32_t qrow = item.q_row0 + row;
         int64_t out_row = -1;  // destination row, or -1 for no real token
         if constexpr (RASTER) {
@@ -618,6 +620,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else if (qrow < p.L) {
           out_row = static_cast<int64_t>(item.bh) * p.L + qrow;
         }
+        // log of the row's sum of exp(scale * s): reference max plus log of the sum
+        // taken against it, from log2 units to natural log
+        if (p.lse != nullptr && h == 0 && out_row >= 0) p.lse[out_row] = (m_run + log2f(l_tot)) * 0.6931471805599453f;
         uint4* dst = reinterpret_cast<uint4*>(p.out + (out_row >= 0 ? out_row : 0) * D + h * (D / 2));
 #pragma unroll 1
         for (int c32 = 0; c32 < D / 64; ++c32) {
@@ -776,6 +781,7 @@ FwdParams make_params(void* out, int32_t heads, const Geometry& g, const DeviceS
   p.scale_log2 = scale * 1.4426950408889634f;
   p.err = err_flag;
   p.limit_ns = limit_ns;
+  p.lse = nullptr;
   return p;
 }
 
@@ -783,12 +789,13 @@ FwdParams make_params(void* out, int32_t heads, const Geometry& g, const DeviceS
 
 cudaError_t launch_attention(const void* q, const void* k, const void* v, void* out, int32_t batch,
                              int32_t heads, int32_t d, const Geometry& g, const DeviceSchedule& s, float scale,
-                             int32_t* err_flag, uint64_t limit_ns, cudaStream_t stream) {
+                             int32_t* err_flag, uint64_t limit_ns, cudaStream_t stream, float* lse) {
   const int64_t bh = static_cast<int64_t>(batch) * heads;
   CUtensorMap tq, tk, tv;
   if (!make_tmap(&tq, q, bh, g.L, d) || !make_tmap(&tk, k, bh, g.L, d) || !make_tmap(&tv, v, bh, g.L, d))
     return cudaErrorInvalidValue;
-  const FwdParams p = make_params(out, heads, g, s, scale, err_flag, limit_ns);
+  FwdParams p = make_params(out, heads, g, s, scale, err_flag, limit_ns);
+  p.lse = lse;
   if (d == 128)
     return s.masked ? launch_d<128, true, false>(tq, tk, tv, p, stream) : launch_d<128, false, false>(tq, tk, tv, p, stream);
   return s.masked ? launch_d<64, true, false>(tq, tk, tv, p, stream) : launch_d<64, false, false>(tq, tk, tv, p, stream);

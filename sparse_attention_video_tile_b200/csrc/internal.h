@@ -64,6 +64,12 @@ void build_schedule(const Geometry& g, int32_t batch, int32_t heads, const sta_d
 void build_schedule_raster(const Geometry& g, int32_t batch, int32_t heads, const sta_dim3* windows,
                            HostSchedule* out);
 
+// The same windows seen from the key side, for the backward pass: one item per
+// (batch, head, block of 128 key rows) with the list of 128-row query blocks that
+// attend it (stored in kv_rows).  Ntile must be a multiple of 128.
+void build_schedule_transposed(const Geometry& g, int32_t batch, int32_t heads, const sta_dim3* windows,
+                               HostSchedule* out);
+
 // Whether a tile splits into 128-row slabs of whole frames (th * tw divides 128 and
 // tt is a multiple of 128 / (th * tw)): the raster-order kernel loads each slab as
 // one TMA box.
@@ -94,11 +100,12 @@ struct DeviceSchedule {
   const uint32_t* kv_masks = nullptr;
 };
 
-// Attention on tiled-order tensors ([BH, L, d]).
+// Attention on tiled-order tensors ([BH, L, d]); lse, when not null, receives
+// each row's log-sum-exp ([BH, L] fp32, tiled order).
 cudaError_t launch_attention(const void* q, const void* k, const void* v, void* out,
                              int32_t batch, int32_t heads, int32_t d, const Geometry& g,
                              const DeviceSchedule& s, float scale, int32_t* err_flag,
-                             uint64_t limit_ns, cudaStream_t stream);
+                             uint64_t limit_ns, cudaStream_t stream, float* lse = nullptr);
 
 // Attention on raster-order tensors ([BH, T, H, W, d]): the tile reorder is done by
 // the TMA loads and the epilogue's addressing; pad tokens read as zeros.
@@ -106,6 +113,15 @@ cudaError_t launch_attention_raster(const void* q, const void* k, const void* v,
                                     int32_t batch, int32_t heads, int32_t d, const Geometry& g,
                                     const DeviceSchedule& s, float scale, int32_t* err_flag,
                                     uint64_t limit_ns, cudaStream_t stream);
+
+// Backward pass on tiled-order tensors: D = rowsum(dout * out) into dvec ([BH, L]
+// fp32 scratch), then dq over the forward schedule and dk, dv over the transposed
+// one (backward.cu).  Ntile must be a multiple of 128.
+cudaError_t launch_backward(const void* q, const void* k, const void* v, const void* out, const void* dout,
+                            const float* lse, float* dvec, void* dq, void* dk, void* dv, int32_t batch,
+                            int32_t heads, int32_t d, const Geometry& g, const DeviceSchedule& fwd,
+                            const DeviceSchedule& tr, float scale, int32_t* err_flag, uint64_t limit_ns,
+                            cudaStream_t stream);
 
 cudaError_t launch_selftest_wait(int32_t* err_flag, uint64_t limit_ns, cudaStream_t stream);
 

@@ -151,6 +151,55 @@ void build_schedule(const Geometry& g, int32_t batch, int32_t heads, const sta_d
                    [](const WorkItem& x, const WorkItem& y) { return x.kv_len > y.kv_len; });
 }
 
+void build_schedule_transposed(const Geometry& g, int32_t batch, int32_t heads, const sta_dim3* windows,
+                               HostSchedule* s) {
+  // Same windows as build_schedule, seen from the key side: key tile c is attended
+  // by the query tiles a whose window contains c.  Only Ntile multiples of 128.
+  s->masked = false;
+  s->items.clear();
+  s->kv_rows.clear();
+  s->head_win.assign(static_cast<size_t>(heads) * 4, 0);
+  s->attended_pairs = 0;
+  const int32_t n_tiles = g.nT * g.nH * g.nW;
+  const int32_t bpt = g.ntile / kBlockRows;
+  const int32_t n_kblocks = n_tiles * bpt;
+  std::map<Eff, std::vector<std::pair<int32_t, int32_t>>> lists;  // per key block: (off, len)
+  std::vector<int32_t> tiles;
+  std::vector<Eff> eff(heads);
+  for (int32_t h = 0; h < heads; ++h) {
+    Eff e{std::min(windows[h].t, g.nT), std::min(windows[h].h, g.nH), std::min(windows[h].w, g.nW)};
+    eff[h] = e;
+    s->head_win[h * 4 + 0] = static_cast<int16_t>(e.t);
+    s->head_win[h * 4 + 1] = static_cast<int16_t>(e.h);
+    s->head_win[h * 4 + 2] = static_cast<int16_t>(e.w);
+    s->attended_pairs += static_cast<int64_t>(batch) * g.L * g.ntile * e.t * e.h * e.w;
+    if (lists.count(e)) continue;
+    std::vector<std::vector<int32_t>> by_key(n_tiles);   // query tiles attending each key tile
+    for (int32_t qt = 0; qt < n_tiles; ++qt) {
+      window_tiles(g, e, qt, &tiles);
+      for (int32_t kt : tiles) by_key[kt].push_back(qt);
+    }
+    std::vector<std::pair<int32_t, int32_t>>& per_kb = lists[e];
+    per_kb.resize(n_kblocks);
+    for (int32_t kt = 0; kt < n_tiles; ++kt) {
+      const int32_t off = static_cast<int32_t>(s->kv_rows.size());
+      for (int32_t qt : by_key[kt])
+        for (int32_t b = 0; b < bpt; ++b) s->kv_rows.push_back(qt * g.ntile + b * kBlockRows);
+      const int32_t len = static_cast<int32_t>(s->kv_rows.size()) - off;
+      for (int32_t b = 0; b < bpt; ++b) per_kb[kt * bpt + b] = {off, len};
+    }
+  }
+  s->items.reserve(static_cast<size_t>(batch) * heads * n_kblocks);
+  for (int32_t b = 0; b < batch; ++b)
+    for (int32_t h = 0; h < heads; ++h) {
+      const auto& per_kb = lists[eff[h]];
+      for (int32_t kb = 0; kb < n_kblocks; ++kb)
+        s->items.push_back(WorkItem{b * heads + h, kb * kBlockRows, per_kb[kb].first, per_kb[kb].second});
+    }
+  std::stable_sort(s->items.begin(), s->items.end(),
+                   [](const WorkItem& x, const WorkItem& y) { return x.kv_len > y.kv_len; });
+}
+
 namespace {
 
 // Whether tiled row m (of the padded latent) is a real token.

@@ -93,6 +93,33 @@ def test_validation_codes(lib):
     assert lib.sta_attended_pairs(1, 1, sta._d3((4, 8, 8)), sta._d3((3, 4, 4)), sta._windows([(1, 1, 1)])) == -1
 
 
+def _call_bwd(lib, base=0x1000000, lse=0x9000000, batch=1, heads=1, d=128, grid=(6, 8, 16), tile=(6, 8, 8),
+              windows=((1, 1, 1),), scale=0.1, **ptrs):
+    # q, k, v, out, dout, dq, dk, dv spaced 1 MB apart (each [1, 1, 768, 128] bf16 = 192 KB)
+    names = ("q", "k", "v", "out", "dout", "dq", "dk", "dv")
+    p = {n: base + i * (1 << 20) for i, n in enumerate(names)}
+    p.update(ptrs)
+    return lib.sta_attention_bwd(p["q"], p["k"], p["v"], p["out"], p["dout"], lse, p["dq"], p["dk"], p["dv"],
+                                 batch, heads, d, sta._d3(grid), sta._d3(tile), sta._windows(windows),
+                                 ctypes.c_float(scale), None)
+
+
+def test_backward_validation_codes(lib):
+    # fake pointers, never dereferenced: validation fails before the device is touched
+    assert _call_bwd(lib, q=None) == 1
+    assert _call_bwd(lib, lse=None) == 1
+    assert _call_bwd(lib, dk=0x1000000 + 5 * (1 << 20) + 8) == 2
+    assert _call_bwd(lib, lse=0x9000004) == 2
+    assert _call_bwd(lib, d=96) == 6
+    assert _call_bwd(lib, grid=(4, 8, 8), tile=(2, 4, 4)) == 4         # 32-token tiles: not a multiple of 128
+    assert _call_bwd(lib, grid=(6, 8, 17)) == 4
+    assert _call_bwd(lib, windows=((0, 1, 1),)) == 5
+    assert _call_bwd(lib, scale=-1.0) == 10
+    assert _call_bwd(lib, dq=0x1000000) == 3                            # dq over q
+    assert _call_bwd(lib, dv=0x1000000 + 5 * (1 << 20)) == 3           # dv over dq
+    assert _call_bwd(lib, lse=0x1000000 + 6 * (1 << 20)) == 3          # lse inside dk
+
+
 def test_no_cpu_fallback_without_gpu(lib):
     import torch
     if torch.cuda.is_available():
@@ -100,3 +127,4 @@ def test_no_cpu_fallback_without_gpu(lib):
     # valid arguments: the library must report a CUDA/architecture error, not compute on the host
     assert _call_reorder(lib, 0x100000, 0x200000) in (7, 8)
     assert _call_attn(lib) in (7, 8)
+    assert _call_bwd(lib) in (7, 8)

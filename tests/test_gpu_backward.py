@@ -1,0 +1,109 @@
+"""GPU parity of the backward pass (through the C ABI) against the fp64 oracle.
+
+The oracle's backward is the chain rule of masked softmax attention, pinned by
+autograd, finite differences and closed forms (oracle_pins.py).  The CUDA path
+takes bf16 operands, accumulates in fp32, rounds P and dS to bf16 for the
+products that take them and rounds dq, dk, dv to bf16.  Each of those roundings
+is a relative error of at most 2^-9 per element, so the relative Frobenius error
+of a gradient is a small multiple of 2^-9 (about 2.4e-3 measured on B200);
+the bounds below allow 5e-3, and for the largest element error 1 % of the
+gradient's largest magnitude.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle.sta_oracle as O
+import workloads as W
+import sparse_attention_video_tile_b200 as sta
+
+pytestmark = pytest.mark.gpu
+
+REL_FRO = 5e-3
+MAX_REL_TO_PEAK = 1e-2
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _device():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from sparse_attention_video_tile_b200.build import build
+    build()
+    sta.load_library()
+    torch.cuda.set_device(0)
+    yield
+    torch.cuda.synchronize()
+
+
+def _gpu_backward(cfg, seed):
+    """Forward (with log-sum-exp) and backward on tiled tensors; gradients returned in
+    raster order, with the raster inputs and output gradient."""
+    q, k, v = W.make_qkv(cfg, seed)
+    do = W.make_qkv(cfg, seed + 100)[0]
+    dev = [x.cuda() for x in (q, k, v, do)]
+    qt, kt, vt, dot = (torch.empty_like(x) for x in dev)
+    for src, dst in zip(dev, (qt, kt, vt, dot)):
+        sta.sta_tile_reorder(src, dst, cfg.grid, cfg.tile)
+    ot = torch.empty_like(qt)
+    lse = torch.empty(cfg.batch, cfg.heads, cfg.L, device="cuda", dtype=torch.float32)
+    sta.sta_attention_fwd_lse(qt, kt, vt, ot, lse, cfg.grid, cfg.tile, cfg.windows, cfg.scale)
+    grads = [torch.full_like(qt, float("nan")) for _ in range(3)]
+    sta.sta_attention_bwd(qt, kt, vt, ot, dot, lse, *grads, cfg.grid, cfg.tile, cfg.windows, cfg.scale)
+    torch.cuda.synchronize()
+    assert sta.sta_check_device_status() == sta.STA_OK
+    raster = []
+    for g in grads:
+        r = torch.empty_like(g)
+        sta.sta_tile_unorder(g, r, cfg.grid, cfg.tile)
+        raster.append(r)
+    torch.cuda.synchronize()
+    return (q, k, v, do), [r.float().cpu().numpy().astype(np.float64) for r in raster]
+
+
+def _compare(got, want, what):
+    assert np.all(np.isfinite(got)), f"{what}: non-finite"
+    rel = np.linalg.norm(got - want) / np.linalg.norm(want)
+    peak = np.abs(want).max()
+    worst = np.abs(got - want).max()
+    assert rel <= REL_FRO, f"{what}: rel Frobenius {rel:.3e}"
+    assert worst <= MAX_REL_TO_PEAK * peak, f"{what}: max abs {worst:.3e} vs peak {peak:.3e}"
+
+
+CASES = [
+    W.CONFIGS["small"],
+    W.custom_config("bwd_b2_d64", 2, 3, 64, (4, 16, 24), (2, 8, 8), [(1, 1, 1), (3, 3, 3), (1, 2, 3)]),
+    W.custom_config("bwd_image", 1, 2, 128, (1, 32, 48), (1, 8, 16), [(1, 3, 3), (1, 4, 2)]),
+    W.custom_config("bwd_dense", 1, 1, 128, (6, 16, 16), (6, 8, 8), [(1, 9, 9)]),   # window covers the grid
+]
+
+
+@pytest.mark.parametrize("cfg", CASES, ids=lambda c: c.name)
+def test_backward_full_parity(cfg):
+    (q, k, v, do), got = _gpu_backward(cfg, seed=5)
+    for b in range(cfg.batch):
+        for h in range(cfg.heads):
+            want = O.sta_attention_backward_head(q[b, h].double().numpy(), k[b, h].double().numpy(),
+                                                 v[b, h].double().numpy(), do[b, h].double().numpy(),
+                                                 cfg.grid, cfg.tile, cfg.windows[h], cfg.scale)
+            for name, g, w in zip(("dq", "dk", "dv"), (x[b, h] for x in got), want):
+                _compare(g, w, f"{cfg.name} b{b} h{h} {name}")
+
+
+def test_backward_hunyuan_sampled_dq_and_sums():
+    """At the full 30x48x80 size: dq of sampled rows (a row's dq needs only its own
+    window), and for dk and dv the closed forms sum_k dv = sum_q dO and
+    sum_k dk = 0, which hold at any size."""
+    cfg = W.CONFIGS["hunyuan"]
+    heads = (0, 13)
+    (q, k, v, do), got = _gpu_backward(cfg, seed=7)
+    rng = np.random.default_rng(3)
+    coords = O.raster_coords(cfg.grid)
+    for h in heads:
+        rows = np.sort(rng.choice(cfg.L, 48, replace=False))
+        q64, k64, v64, do64 = (x[0, h].double().numpy() for x in (q, k, v, do))
+        mask = O.sta_mask(coords[rows], coords, cfg.grid, cfg.tile, cfg.windows[h])
+        want_dq, _, _ = O.masked_softmax_attention_backward(q64[rows], k64, v64, mask, cfg.scale, do64[rows])
+        _compare(got[0][0, h][rows], want_dq, f"hunyuan h{h} dq rows")
+        dv_sum, do_sum = got[2][0, h].sum(axis=0), do64.sum(axis=0)
+        assert np.abs(dv_sum - do_sum).max() <= 1e-2 * np.abs(do_sum).max() + 0.5
+        assert np.abs(got[1][0, h].sum(axis=0)).max() <= 1e-2 * np.abs(got[1][0, h]).sum(axis=0).max() + 0.5

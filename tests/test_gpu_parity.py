@@ -119,6 +119,38 @@ def test_attention_padded_latents(cfg):
     _full_parity(cfg, seed=6, pad=True)
 
 
+LSE_ABS = 1e-3   # fp32 scores from bf16 inputs, MUFU exponentials, fp32 sums: about 1e-5 expected
+
+
+@pytest.mark.parametrize("name", ["tiny", "small", "batch2_perhead"])
+def test_attention_lse(name):
+    """The forward's per-row log-sum-exp against the oracle's, and the output
+    unchanged by asking for it."""
+    cfg = W.CONFIGS[name] if name in W.CONFIGS else \
+        W.custom_config(name, 2, 3, 128, (4, 16, 24), (2, 8, 8), [(1, 1, 1), (3, 3, 3), (1, 2, 3)])
+    q, k, v = W.make_qkv(cfg, 4)
+    qd, kd, vd = (x.cuda() for x in (q, k, v))
+    qt, kt, vt = (torch.empty_like(x) for x in (qd, kd, vd))
+    for src, dst in ((qd, qt), (kd, kt), (vd, vt)):
+        sta.sta_tile_reorder(src, dst, cfg.grid, cfg.tile)
+    o1, o2 = torch.empty_like(qt), torch.empty_like(qt)
+    lse = torch.full((cfg.batch, cfg.heads, cfg.L), float("nan"), device="cuda", dtype=torch.float32)
+    sta.sta_attention_fwd(qt, kt, vt, o1, cfg.grid, cfg.tile, cfg.windows, cfg.scale)
+    sta.sta_attention_fwd_lse(qt, kt, vt, o2, lse, cfg.grid, cfg.tile, cfg.windows, cfg.scale)
+    torch.cuda.synchronize()
+    assert sta.sta_check_device_status() == sta.STA_OK
+    assert torch.equal(o1, o2)
+    tiled = O.tiled_of_raster(cfg.grid, cfg.tile)   # raster token n -> tiled row
+    got = lse.cpu().numpy().astype(np.float64)
+    for b in range(cfg.batch):
+        for h in range(cfg.heads):
+            want = O.sta_lse_head(q[b, h].double().numpy(), k[b, h].double().numpy(), cfg.grid, cfg.tile,
+                                  cfg.windows[h], cfg.scale)
+            err = np.abs(got[b, h][tiled] - want)
+            assert np.all(np.isfinite(got[b, h])), f"{name} b{b} h{h}: non-finite lse"
+            assert err.max() <= LSE_ABS, f"{name} b{b} h{h}: lse max abs {err.max():.3e}"
+
+
 def test_attention_tiny_other_seeds():
     for seed in (1, 2):
         _full_parity(W.CONFIGS["tiny"], seed)
