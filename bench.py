@@ -39,7 +39,7 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # workload, from the ncu capture summarised in profiles/sta_fwd_kernel_hunyuan_4heads.md (4-head
 # case, scaled by 6 to 24 heads: traffic is per head).  Valid only for the kernel source it was
 # taken on.
-PROFILED_TRAFFIC = {"sha1": "06ba0203e5df56d358c6f7b6a3e71d125a4bdfd9", "bytes_per_launch": 6 * (361.18272e6 + 104.259328e6),
+PROFILED_TRAFFIC = {"sha1": "b8305f495bbde1d2b28800bbb7d3bedbc235e120", "bytes_per_launch": 6 * (362.627072e6 + 106.815232e6),
                     "workload": "hunyuan"}
 
 
