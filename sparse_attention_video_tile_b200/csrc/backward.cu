@@ -15,16 +15,18 @@
 // its window), and dK, dV over the transposed items (a 128-row key block and the
 // query blocks whose windows contain it).  Each attention kernel is one CTA per SM:
 //
-//   * warp 4 loads the item's fixed operands (Q and dO, or K and V) and streams
+//   * warp 8 loads the item's fixed operands (Q and dO, or K and V) and streams
 //     the per-block operands (K and V, or Q and dO, plus lse and D of the query
 //     block) through a two-stage shared-memory ring with TMA;
-//   * warp 5 issues the tcgen05 MMAs from one thread: S and dP (both operands in
+//   * warp 9 issues the tcgen05 MMAs from one thread: S and dP (both operands in
 //     shared memory, fp32 in TMEM), then after the elementwise step the
 //     accumulations with the bf16 P and dS read from TMEM (dQ += dS K, or
 //     dV += P^T dO and dK += dS^T Q);
-//   * warps 0-3, one TMEM lane (row) per thread, turn S and dP into P and dS and
-//     write them back to TMEM as bf16 over the first columns of S and dP, and at
-//     the end of an item scale and store the accumulators as bf16 rows.
+//   * warps 0-7 turn S and dP into P and dS: TMEM lane = row, warps w and w+4
+//     take columns 0-63 and 64-127 of the rows of lane quadrant w, and each writes
+//     its P and dS back to TMEM as bf16 over the first 32 of its own columns of S
+//     and dP (so neither overwrites columns the other still reads).  At the end of
+//     an item each warp scales and stores its half of the accumulators' columns.
 //
 // Tiles must be multiples of 128 rows, so every block pair in a schedule is fully
 // attended and no mask exists.  Every wait is bounded (see ptx.cuh).
@@ -43,9 +45,9 @@ namespace {
 
 using namespace ptx;
 
-constexpr int kBwdThreads = 192;   // warps 0-3 elementwise + epilogue, 4 producer, 5 MMA issuer
-constexpr int kBwdProducer = 4;
-constexpr int kBwdMma = 5;
+constexpr int kBwdThreads = 320;   // warps 0-7 elementwise + epilogue, 8 producer, 9 MMA issuer
+constexpr int kBwdProducer = 8;
+constexpr int kBwdMma = 9;
 constexpr int kBwdTmemCols = 512;  // S at 0, dP at 128, accumulators at 256 (and 384)
 
 enum BwdKind { kDq = 0, kDkDv = 1 };
@@ -130,7 +132,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(sb + S::kKvEmpty + 8 * s, 1);
     }
     mbar_init(sb + S::kSFull, 1);
-    mbar_init(sb + S::kPFull, 4);   // one arrival per elementwise warp
+    mbar_init(sb + S::kPFull, 8);   // one arrival per elementwise warp
     mbar_init(sb + S::kOFull, 1);
     mbar_init(sb + S::kDrain, 1);
     *abort_flag = 0;
@@ -233,22 +235,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           if (!ok) break;
           tc_fence_after();
           // accumulations: B operands are the streamed blocks read MN-major (rows = K
-          // dimension, 16 rows = 2 KB per slice); A is bf16 in TMEM (8 columns per slice)
+          // dimension, 16 rows = 2 KB per slice); A is bf16 in TMEM (8 columns per
+          // slice), keys 0-63 in columns 0-31 and keys 64-127 in columns 64-95
           const uint64_t dm0 = sdesc_sw128(base, kBlockRows * 128, 1024);
           const uint64_t dm1 = sdesc_sw128(base + kBlockBytes, kBlockRows * 128, 1024);
           if (KIND == kDq) {
             // dQ += dS K
 #pragma unroll
             for (int k16 = 0; k16 < 8; ++k16)
-              umma_ts(tA0, tS + k16 * 8, dm0 + static_cast<uint64_t>(k16 * (2048 >> 4)), idesc_ts, (j > 0 || k16 > 0));
+              umma_ts(tA0, tS + (k16 >> 2) * 64 + (k16 & 3) * 8, dm0 + static_cast<uint64_t>(k16 * (2048 >> 4)), idesc_ts,
+                      (j > 0 || k16 > 0));
           } else {
             // dV += P^T dO, dK += dS^T Q
 #pragma unroll
             for (int k16 = 0; k16 < 8; ++k16)
-              umma_ts(tA0, tS + k16 * 8, dm1 + static_cast<uint64_t>(k16 * (2048 >> 4)), idesc_ts, (j > 0 || k16 > 0));
+              umma_ts(tA0, tS + (k16 >> 2) * 64 + (k16 & 3) * 8, dm1 + static_cast<uint64_t>(k16 * (2048 >> 4)), idesc_ts,
+                      (j > 0 || k16 > 0));
 #pragma unroll
             for (int k16 = 0; k16 < 8; ++k16)
-              umma_ts(tA1, tP + k16 * 8, dm0 + static_cast<uint64_t>(k16 * (2048 >> 4)), idesc_ts, (j > 0 || k16 > 0));
+              umma_ts(tA1, tP + (k16 >> 2) * 64 + (k16 & 3) * 8, dm0 + static_cast<uint64_t>(k16 * (2048 >> 4)), idesc_ts,
+                      (j > 0 || k16 > 0));
           }
           umma_commit(sb + S::kKvEmpty + 8 * st);
           if (j + 1 == n) {
@@ -263,9 +269,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ elementwise + epilogue
-    const int row = warp * 32 + lane;   // TMEM lane = row of the item's block
-    const uint32_t tl = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    const uint32_t tS = tl, tP = tl + 128, tA0 = tl + 256, tA1 = tl + 384;
+    const int quad = warp & 3, hh = warp >> 2;   // lane quadrant; columns [64 hh, 64 hh + 64)
+    const int row = quad * 32 + lane;             // TMEM lane = row of the item's block
+    const uint32_t tl = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    const uint32_t tS = tl + 64 * hh, tP = tl + 128 + 64 * hh, tA0 = tl + 256, tA1 = tl + 384;
     const float sl2 = p.scale_log2;
     constexpr float kLog2e = 1.4426950408889634f;
     uint32_t seq = 0, blk = 0;
@@ -290,28 +297,41 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           if (!ok) break;
         }
         tc_fence_after();
-        const float* col_lse = reinterpret_cast<const float*>(smem + S::kStage0 + st * S::kStageBytes + 2 * kBlockBytes);
-        const float* col_d = col_lse + 128;
+        // lse and D of this warp's 64 columns (dK, dV kernel), read four at a time
+        const float4* col_lse4 = reinterpret_cast<const float4*>(smem + S::kStage0 + st * S::kStageBytes +
+                                                                 2 * kBlockBytes) + 16 * hh;
+        const float4* col_d4 = col_lse4 + 32;
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
           uint32_t s32[32], p32[32];
           tmem_ld32(tS + 32 * c, s32);
           tmem_ld32(tP + 32 * c, p32);
           tmem_wait_ld();
           uint32_t pk[16], dk[16];
 #pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            float pr[2], dsv[2];
+          for (int i = 0; i < 32; i += 4) {
+            float l2[4], dd[4];
+            if (KIND == kDq) {
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              const int col = 32 * c + i + u;
-              const float l2 = KIND == kDq ? lse2_row : col_lse[col] * kLog2e;
-              const float dd = KIND == kDq ? d_row : col_d[col];
-              pr[u] = ex2_approx(fmaf(__uint_as_float(s32[i + u]), sl2, -l2));
-              dsv[u] = pr[u] * (__uint_as_float(p32[i + u]) - dd);
+              for (int u = 0; u < 4; ++u) {
+                l2[u] = lse2_row;
+                dd[u] = d_row;
+              }
+            } else {
+              const float4 lv = col_lse4[8 * c + i / 4], dv4 = col_d4[8 * c + i / 4];
+              l2[0] = lv.x * kLog2e; l2[1] = lv.y * kLog2e; l2[2] = lv.z * kLog2e; l2[3] = lv.w * kLog2e;
+              dd[0] = dv4.x; dd[1] = dv4.y; dd[2] = dv4.z; dd[3] = dv4.w;
+            }
+            float pr[4], dsv[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              pr[u] = ex2_approx(fmaf(__uint_as_float(s32[i + u]), sl2, -l2[u]));
+              dsv[u] = pr[u] * (__uint_as_float(p32[i + u]) - dd[u]);
             }
             pk[i >> 1] = pack_bf16x2(pr[0], pr[1]);
+            pk[(i >> 1) + 1] = pack_bf16x2(pr[2], pr[3]);
             dk[i >> 1] = pack_bf16x2(dsv[0], dsv[1]);
+            dk[(i >> 1) + 1] = pack_bf16x2(dsv[2], dsv[3]);
           }
           if (KIND == kDq) {
             tmem_st16(tS + 16 * c, dk);    // dS over S
@@ -331,13 +351,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (!ok) break;
       tc_fence_after();
       for (int a = 0; a < (KIND == kDq ? 1 : 2); ++a) {
-        const uint32_t tacc = a == 0 ? tA0 : tA1;
+        // this warp's half of the accumulator's columns
+        const uint32_t tacc = (a == 0 ? tA0 : tA1) + hh * (D / 2);
         // dQ (a = 0) and dK (a = 1 of dK, dV) carry the softmax scale; dV does not
         const float mul = (KIND == kDq || a == 1) ? p.scale : 1.0f;
         __nv_bfloat16* dst_t = KIND == kDq ? p.out0 : (a == 0 ? p.out1 : p.out0);
-        uint4* dst = reinterpret_cast<uint4*>(dst_t + grow * D);
+        uint4* dst = reinterpret_cast<uint4*>(dst_t + grow * D + hh * (D / 2));
 #pragma unroll 1
-        for (int c32 = 0; c32 < D / 32; ++c32) {
+        for (int c32 = 0; c32 < D / 64; ++c32) {
           uint32_t o[32];
           tmem_ld32(tacc + 32 * c32, o);
           tmem_wait_ld();
