@@ -82,6 +82,21 @@ int64_t sta_attended_pairs(int32_t batch, int32_t heads, sta_dim3 grid, sta_dim3
                            const sta_dim3* windows);
 
 /*
+ * The (query block, key block) pairs of the work schedules (host only), so that
+ * they can be checked against the window rule without a GPU: the forward's
+ * schedule (transposed = 0: each 128-row query block with the 128-row key blocks
+ * of its window) or the backward's key-side schedule (transposed = 1: each key
+ * block with the query blocks whose windows contain it).  Up to `capacity`
+ * triples (batch * heads + head, first tiled row of the query block, first tiled
+ * row of the key block) are written to `out` (host int32[3 * capacity], may be
+ * NULL); returns the number of pairs, or -1 on an invalid argument or a tile
+ * that does not hold a multiple of 128 tokens.  No device is touched.
+ */
+int64_t sta_schedule_block_pairs(int32_t batch, int32_t heads, sta_dim3 grid, sta_dim3 tile,
+                                 const sta_dim3* windows, int32_t transposed, int32_t* out,
+                                 int64_t capacity);
+
+/*
  * Reorder raster -> tiled (summary page, "Method details": tokens of a tile made
  * contiguous).  src, dst: device bf16 [batch_heads, L, d], 16-byte aligned, not
  * overlapping.  dst[bh, tiled(n), :] = src[bh, n, :], bit-exact.

@@ -56,6 +56,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "sta_last_cuda_error": (ctypes.c_char_p, []),
         "sta_tile_index_map": (ctypes.c_int, [D3, D3, ctypes.POINTER(ctypes.c_int32)]),
         "sta_attended_pairs": (I64, [I32, I32, D3, D3, ctypes.POINTER(D3)]),
+        "sta_schedule_block_pairs": (I64, [I32, I32, D3, D3, ctypes.POINTER(D3), I32, ctypes.POINTER(ctypes.c_int32), I64]),
         "sta_tile_reorder": (ctypes.c_int, [P, P, I64, I32, D3, D3, P]),
         "sta_tile_unorder": (ctypes.c_int, [P, P, I64, I32, D3, D3, P]),
         "sta_attention_fwd": (ctypes.c_int, [P, P, P, P, I32, I32, I32, D3, D3, ctypes.POINTER(D3), F, P]),
@@ -137,6 +138,19 @@ def sta_attended_pairs(batch: int, heads: int, grid, tile, windows) -> int:
     if r < 0:
         raise StaError(10, "sta_attended_pairs")
     return int(r)
+
+
+def sta_schedule_block_pairs(batch: int, heads: int, grid, tile, windows, transposed: bool = False) -> np.ndarray:
+    """(bh, query block row, key block row) of every block pair of the forward's
+    schedule or, with ``transposed``, of the backward's key-side schedule (host only)."""
+    lib = load_library()
+    args = (int(batch), int(heads), _d3(grid), _d3(tile), _windows(windows), int(bool(transposed)))
+    n = lib.sta_schedule_block_pairs(*args, None, 0)
+    if n < 0:
+        raise StaError(10, "sta_schedule_block_pairs")
+    out = np.empty((max(n, 1), 3), dtype=np.int32)
+    lib.sta_schedule_block_pairs(*args, out.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), n)
+    return out[:n]
 
 
 def sta_tile_reorder(src, dst, grid, tile, stream=None) -> None:

@@ -223,6 +223,30 @@ int64_t sta_attended_pairs(int32_t batch, int32_t heads, sta_dim3 grid, sta_dim3
   return total * batch;
 }
 
+int64_t sta_schedule_block_pairs(int32_t batch, int32_t heads, sta_dim3 grid, sta_dim3 tile,
+                                 const sta_dim3* windows, int32_t transposed, int32_t* out, int64_t capacity) {
+  Geometry g;
+  if (make_geometry(grid, tile, &g) != STA_OK || batch < 1 || heads < 1 || !windows || capacity < 0) return -1;
+  if (g.ntile % kBlockRows != 0) return -1;
+  for (int32_t h = 0; h < heads; ++h)
+    if (windows[h].t < 1 || windows[h].h < 1 || windows[h].w < 1) return -1;
+  HostSchedule hs;
+  if (transposed)
+    build_schedule_transposed(g, batch, heads, windows, &hs);
+  else
+    build_schedule(g, batch, heads, windows, &hs);
+  int64_t n = 0;
+  for (const WorkItem& it : hs.items)
+    for (int32_t j = 0; j < it.kv_len; ++j, ++n) {
+      if (!out || n >= capacity) continue;
+      const int32_t listed = hs.kv_rows[it.kv_off + j];
+      out[3 * n + 0] = it.bh;
+      out[3 * n + 1] = transposed ? listed : it.q_row0;   // query block
+      out[3 * n + 2] = transposed ? it.q_row0 : listed;   // key block
+    }
+  return n;
+}
+
 sta_status sta_tile_reorder(const void* src, void* dst, int64_t batch_heads, int32_t d, sta_dim3 grid,
                             sta_dim3 tile, void* stream) {
   Geometry g;

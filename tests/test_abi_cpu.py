@@ -11,6 +11,7 @@ import numpy as np
 import pytest
 
 import oracle.sta_oracle as O
+import workloads as W
 from workloads import CONFIGS
 
 import sparse_attention_video_tile_b200 as sta
@@ -128,3 +129,42 @@ def test_no_cpu_fallback_without_gpu(lib):
     assert _call_reorder(lib, 0x100000, 0x200000) in (7, 8)
     assert _call_attn(lib) in (7, 8)
     assert _call_bwd(lib) in (7, 8)
+
+
+SCHEDULE_CASES = [
+    ("small", None),
+    ("b2_perhead", W.custom_config("b2_perhead", 2, 3, 64, (4, 16, 24), (2, 8, 8), [(1, 1, 1), (3, 3, 3), (1, 2, 3)])),
+    ("image", W.custom_config("image", 1, 2, 128, (1, 32, 48), (1, 8, 16), [(1, 3, 3), (1, 4, 2)])),
+    ("even", W.custom_config("even", 1, 1, 128, (6, 32, 32), (2, 8, 8), [(2, 2, 4)])),
+]
+
+
+@pytest.mark.parametrize("name,cfg", SCHEDULE_CASES, ids=[c[0] for c in SCHEDULE_CASES])
+def test_schedules_cover_exactly_the_window_blocks(lib, name, cfg):
+    """Both work schedules (forward: query blocks with their key blocks; backward:
+    key blocks with their query blocks) hold exactly the block pairs whose tiles the
+    oracle's window rule connects, each once."""
+    cfg = cfg or W.CONFIGS[name]
+    tiled = O.tiled_of_raster(cfg.grid, cfg.tile)
+    raster_of_tiled = np.empty_like(tiled)
+    raster_of_tiled[tiled] = np.arange(tiled.size)
+    coords = O.raster_coords(cfg.grid)
+    nblk = cfg.L // 128
+    rep = coords[raster_of_tiled[np.arange(nblk) * 128]]       # one token of each 128-row block
+    want = set()
+    for b in range(cfg.batch):
+        for h in range(cfg.heads):
+            m = O.sta_mask(rep, rep, cfg.grid, cfg.tile, cfg.windows[h])
+            qi, ki = np.nonzero(m)
+            want.update(zip([b * cfg.heads + h] * len(qi), (qi * 128).tolist(), (ki * 128).tolist()))
+    for transposed in (False, True):
+        got = sta.sta_schedule_block_pairs(cfg.batch, cfg.heads, cfg.grid, cfg.tile, cfg.windows, transposed)
+        triples = list(map(tuple, got.tolist()))
+        assert len(triples) == len(set(triples)), "a block pair appears twice"
+        assert set(triples) == want
+        assert len(triples) * 128 * 128 == O.attended_pairs(cfg.batch, cfg.grid, cfg.tile, cfg.windows)
+
+
+def test_schedule_pairs_reject_small_tiles(lib):
+    assert lib.sta_schedule_block_pairs(1, 1, sta._d3((4, 8, 8)), sta._d3((2, 4, 4)), sta._windows([(1, 1, 1)]),
+                                        0, None, 0) == -1
