@@ -321,3 +321,60 @@ def sta_forward(q, k, v, grid, tile, window_per_head, scale: Optional[float] = N
     sta_attention_fwd(qt, kt, vt, ot, grid, tile, window_per_head, scale, stream)
     sta_tile_unorder(ot, out, grid, tile, stream)
     return out
+
+
+def sta_forward_from_host(q_h, k_h, v_h, out_h, grid, tile, window_per_head, scale: Optional[float] = None,
+                          heads_per_chunk: int = 4, device=None) -> None:
+    """STA forward from pinned host tensors [B, heads, L, d] (bf16, raster order)
+    into the pinned host tensor ``out_h``, with the copies overlapped with the
+    computation: heads go through in chunks, and while one chunk is computed
+    (``sta_forward``) the next is copied in and the previous one copied out, on
+    three CUDA streams.  Per head the result equals ``sta_forward`` on device
+    tensors: heads are independent.  Returns once ``out_h`` holds the output."""
+    import torch
+    if q_h.dim() != 4:
+        raise ValueError("q must be [batch, heads, L, d]")
+    for name, t in (("k", k_h), ("v", v_h), ("out", out_h)):
+        if tuple(t.shape) != tuple(q_h.shape):
+            raise ValueError(f"{name} shape {tuple(t.shape)} differs from q {tuple(q_h.shape)}")
+    for name, t in (("q", q_h), ("k", k_h), ("v", v_h), ("out", out_h)):
+        if t.is_cuda or not t.is_pinned() or not t.is_contiguous() or t.dtype != torch.bfloat16:
+            raise ValueError(f"{name} must be a contiguous pinned host bf16 tensor")
+    B, Hn = int(q_h.shape[0]), int(q_h.shape[1])
+    if len(window_per_head) != Hn:
+        raise ValueError("one window per head is required")
+    if heads_per_chunk < 1:
+        raise ValueError("heads_per_chunk must be positive")
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    chunks = [(b, h0, min(Hn, h0 + heads_per_chunk)) for b in range(B) for h0 in range(0, Hn, heads_per_chunk)]
+    s_in, s_run, s_out = (torch.cuda.Stream(device=dev) for _ in range(3))
+    shape = (1, heads_per_chunk) + tuple(q_h.shape[2:])
+    bufs = [[torch.empty(shape, dtype=q_h.dtype, device=dev) for _ in range(3)] for _ in range(2)]
+    outs = [None, None]
+    copied, computed, drained = ([None, None] for _ in range(3))
+    for i, (b, h0, h1) in enumerate(chunks):
+        slot, n = i % 2, h1 - h0
+        with torch.cuda.stream(s_in):
+            if drained[slot] is not None:
+                s_in.wait_event(computed[slot])       # the slot's inputs are no longer read
+            for buf, src in zip(bufs[slot], (q_h, k_h, v_h)):
+                buf[:, :n].copy_(src[b:b + 1, h0:h1], non_blocking=True)
+            copied[slot] = torch.cuda.Event()
+            copied[slot].record(s_in)
+        with torch.cuda.stream(s_run):
+            s_run.wait_event(copied[slot])
+            if drained[slot] is not None:
+                s_run.wait_event(drained[slot])       # the slot's previous output has been copied out
+            q, k, v = (buf[:, :n] if n == heads_per_chunk else buf[:, :n].contiguous() for buf in bufs[slot])
+            outs[slot] = sta_forward(q, k, v, grid, tile, list(window_per_head[h0:h1]), scale, s_run)
+            computed[slot] = torch.cuda.Event()
+            computed[slot].record(s_run)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(computed[slot])
+            outs[slot].record_stream(s_out)       # its memory is reused only after this copy
+            out_h[b:b + 1, h0:h1].copy_(outs[slot], non_blocking=True)
+            drained[slot] = torch.cuda.Event()
+            drained[slot].record(s_out)
+    s_out.synchronize()
+    s_run.synchronize()
+

@@ -319,3 +319,16 @@ def test_bounded_wait_gives_up_and_context_survives():
     # the flag is cleared and the library still computes correctly
     assert sta.sta_check_device_status() == sta.STA_OK
     _full_parity(W.CONFIGS["tiny"])
+
+
+def test_forward_from_host_equals_device_forward():
+    """The copy-overlapped host entry gives, head by head, the device forward's bits."""
+    cfg = W.custom_config("host_b2", 2, 5, 128, (12, 24, 40), (6, 8, 8),
+                          [(1, 3, 3), (3, 3, 3), (1, 1, 1), (3, 5, 5), (1, 3, 3)])
+    q, k, v = W.make_qkv(cfg, 12)
+    want = sta.sta_forward(q.cuda(), k.cuda(), v.cuda(), cfg.grid, cfg.tile, cfg.windows, cfg.scale)
+    qh, kh, vh = (x.pin_memory() for x in (q, k, v))
+    out_h = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+    sta.sta_forward_from_host(qh, kh, vh, out_h, cfg.grid, cfg.tile, cfg.windows, cfg.scale, heads_per_chunk=2)
+    assert sta.sta_check_device_status() == sta.STA_OK
+    assert torch.equal(out_h, want.cpu())
