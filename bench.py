@@ -388,6 +388,32 @@ def run_ours(args, cfg):
                             "in both the dQ and the dK/dV pass (14 d executed)"}
         del lse, dot, grads
 
+    # ---- the token-major reorders (not part of `value`): [B, L, heads, d] raster
+    # <-> [B, heads, L, d] tiled, the transposes folded into the tile reorder;
+    # algorithmic bytes: one read and one write of the tensor
+    token_major = None
+    if args.aux_steps > 0:
+        tok = out.view(cfg.batch, cfg.L, cfg.heads, cfg.d)   # any bf16 data serves
+        for _ in range(2):
+            sta.sta_tile_reorder_tokens(tok, qt, grid, tile, stream)
+            sta.sta_tile_unorder_tokens(qt, tok, grid, tile, stream)
+        torch.cuda.synchronize()
+        t0, t1, t2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        t0.record(stream)
+        for _ in range(args.aux_steps):
+            sta.sta_tile_reorder_tokens(tok, qt, grid, tile, stream)
+        t1.record(stream)
+        for _ in range(args.aux_steps):
+            sta.sta_tile_unorder_tokens(qt, tok, grid, tile, stream)
+        t2.record(stream)
+        torch.cuda.synchronize()
+        r_ms, u_ms = t0.elapsed_time(t1) / args.aux_steps, t1.elapsed_time(t2) / args.aux_steps
+        r_gbs, u_gbs = (2 * tensor_bytes / (m * 1e-3) / 1e9 for m in (r_ms, u_ms))
+        token_major = {"steps": args.aux_steps, "reorder_ms": r_ms, "reorder_gbs": r_gbs,
+                       "reorder_frac_hbm": r_gbs / hbm, "unorder_ms": u_ms, "unorder_gbs": u_gbs,
+                       "unorder_frac_hbm": u_gbs / hbm}
+        del tok
+
     # ---- end to end through the public API with host buffers
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
     barrier()
@@ -430,7 +456,8 @@ def run_ours(args, cfg):
         "kernels": {"attention_ms": att_ms, "attention_tflops": att_tflops,
                     "path": "fused raster-order kernel, 1 launch per step" if fused else
                             "reorder x3 + tiled attention + unorder, 5 launches per step",
-                    "three_call_path": three, "fused_path": other, "backward": backward},
+                    "three_call_path": three, "fused_path": other, "backward": backward,
+                    "token_major_reorder": token_major},
         "cpu_baseline": cpu,
         "e2e": {"value": job_tflops(world, flops, e2e_ms), "unit": "TFLOPS", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": 3 * tensor_bytes, "d2h_bytes_per_step": tensor_bytes,

@@ -111,6 +111,24 @@ sta_status sta_tile_unorder(const void* src, void* dst, int64_t batch_heads, int
                             sta_dim3 grid, sta_dim3 tile, void* stream);
 
 /*
+ * Reorder with a token-major raster side (summary page, "Method details": the
+ * same tile order): src is device bf16 [batch, L, heads, d] in raster order,
+ * the layout of a [batch, L, heads * d] projection; dst is device bf16
+ * [batch, heads, L, d] in tiled order, as sta_attention_fwd takes it.
+ *   dst[b, h, tiled(n), :] = src[b, n, h, :], bit-exact.
+ * Both 16-byte aligned, not overlapping.  batch = 0 or heads = 0 is a no-op.
+ * Errors: NULL, ALIGN, ALIAS, SHAPE, HEADDIM, ARG (negative batch or heads),
+ * ARCH, CUDA.
+ */
+sta_status sta_tile_reorder_tokens(const void* src, void* dst, int32_t batch, int32_t heads, int32_t d,
+                                   sta_dim3 grid, sta_dim3 tile, void* stream);
+
+/* Inverse of sta_tile_reorder_tokens: src tiled [batch, heads, L, d], dst
+ * token-major raster [batch, L, heads, d]; dst[b, n, h, :] = src[b, h, tiled(n), :]. */
+sta_status sta_tile_unorder_tokens(const void* src, void* dst, int32_t batch, int32_t heads, int32_t d,
+                                   sta_dim3 grid, sta_dim3 tile, void* stream);
+
+/*
  * STA forward on tiled-order tensors (abstract; "Method details"; "Core
  * innovation"): for every head h and query token i,
  *   out[i] = sum_j softmax_j(scale * q_i . k_j) v_j

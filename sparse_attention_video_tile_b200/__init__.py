@@ -59,6 +59,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "sta_schedule_block_pairs": (I64, [I32, I32, D3, D3, ctypes.POINTER(D3), I32, ctypes.POINTER(ctypes.c_int32), I64]),
         "sta_tile_reorder": (ctypes.c_int, [P, P, I64, I32, D3, D3, P]),
         "sta_tile_unorder": (ctypes.c_int, [P, P, I64, I32, D3, D3, P]),
+        "sta_tile_reorder_tokens": (ctypes.c_int, [P, P, I32, I32, I32, D3, D3, P]),
+        "sta_tile_unorder_tokens": (ctypes.c_int, [P, P, I32, I32, I32, D3, D3, P]),
         "sta_attention_fwd": (ctypes.c_int, [P, P, P, P, I32, I32, I32, D3, D3, ctypes.POINTER(D3), F, P]),
         "sta_attention_fwd_raster": (ctypes.c_int, [P, P, P, P, I32, I32, I32, D3, D3, ctypes.POINTER(D3), F, P]),
         "sta_attention_fwd_lse": (ctypes.c_int, [P, P, P, P, P, I32, I32, I32, D3, D3, ctypes.POINTER(D3), F, P]),
@@ -173,6 +175,35 @@ def sta_tile_unorder(src, dst, grid, tile, stream=None) -> None:
     st = load_library().sta_tile_unorder(_tensor_ptr(src, "src"), _tensor_ptr(dst, "dst"), bh, d,
                                          _d3(grid), _d3(tile), _stream(stream))
     _check(st, "sta_tile_unorder")
+
+
+def _token_shapes(tokens, tiled, where: str):
+    """(batch, heads, d) of a token-major [B, L, heads, d] tensor and its tiled
+    [B, heads, L, d] counterpart."""
+    if tokens.dim() != 4 or tiled.dim() != 4:
+        raise ValueError(f"{where}: expected 4-D tensors")
+    b, n, h, d = (int(x) for x in tokens.shape)
+    if tuple(tiled.shape) != (b, h, n, d):
+        raise ValueError(f"{where}: token-major {tuple(tokens.shape)} does not match tiled {tuple(tiled.shape)}")
+    return b, h, d
+
+
+def sta_tile_reorder_tokens(src, dst, grid, tile, stream=None) -> None:
+    """dst[b, h, tiled(n), :] = src[b, n, h, :]: token-major raster [B, L, heads, d]
+    (a [B, L, heads * d] projection viewed per head) to tiled [B, heads, L, d]."""
+    b, h, d = _token_shapes(src, dst, "sta_tile_reorder_tokens")
+    st = load_library().sta_tile_reorder_tokens(_tensor_ptr(src, "src"), _tensor_ptr(dst, "dst"), b, h, d,
+                                                _d3(grid), _d3(tile), _stream(stream))
+    _check(st, "sta_tile_reorder_tokens")
+
+
+def sta_tile_unorder_tokens(src, dst, grid, tile, stream=None) -> None:
+    """dst[b, n, h, :] = src[b, h, tiled(n), :]: tiled [B, heads, L, d] to
+    token-major raster [B, L, heads, d]."""
+    b, h, d = _token_shapes(dst, src, "sta_tile_unorder_tokens")
+    st = load_library().sta_tile_unorder_tokens(_tensor_ptr(src, "src"), _tensor_ptr(dst, "dst"), b, h, d,
+                                                _d3(grid), _d3(tile), _stream(stream))
+    _check(st, "sta_tile_unorder_tokens")
 
 
 def sta_attention_fwd(q, k, v, out, grid, tile, window_per_head, scale: float, stream=None) -> None:
@@ -320,6 +351,30 @@ def sta_forward(q, k, v, grid, tile, window_per_head, scale: Optional[float] = N
     sta_tile_reorder(v, vt, grid, tile, stream)
     sta_attention_fwd(qt, kt, vt, ot, grid, tile, window_per_head, scale, stream)
     sta_tile_unorder(ot, out, grid, tile, stream)
+    return out
+
+
+def sta_forward_tokens(q, k, v, grid, tile, window_per_head, scale: Optional[float] = None,
+                       stream=None, workspace: Optional[Tuple] = None):
+    """Full STA forward on token-major raster [B, L, heads, d] bf16 CUDA tensors
+    (the layout of per-head views of [B, L, heads * d] projections), output in the
+    same layout.  The transposes to and from [B, heads, L, d] are part of the tile
+    reorders (``sta_tile_reorder_tokens`` / ``sta_tile_unorder_tokens``), so there
+    is no extra pass over memory.  The grid must be a tile multiple.
+    ``workspace`` may hold four preallocated tiled [B, heads, L, d] tensors."""
+    import torch
+    if scale is None:
+        scale = 1.0 / float(q.shape[-1]) ** 0.5
+    b, n, h, d = (int(x) for x in q.shape)
+    if workspace is None:
+        workspace = tuple(torch.empty((b, h, n, d), dtype=q.dtype, device=q.device) for _ in range(4))
+    qt, kt, vt, ot = workspace
+    sta_tile_reorder_tokens(q, qt, grid, tile, stream)
+    sta_tile_reorder_tokens(k, kt, grid, tile, stream)
+    sta_tile_reorder_tokens(v, vt, grid, tile, stream)
+    sta_attention_fwd(qt, kt, vt, ot, grid, tile, window_per_head, scale, stream)
+    out = torch.empty_like(q)
+    sta_tile_unorder_tokens(ot, out, grid, tile, stream)
     return out
 
 

@@ -268,6 +268,32 @@ sta_status sta_tile_unorder(const void* src, void* dst, int64_t batch_heads, int
 }
 
 namespace {
+// sta_tile_reorder_tokens and sta_tile_unorder_tokens: validation, launch.
+sta_status reorder_tokens_impl(const void* src, void* dst, int32_t batch, int32_t heads, int32_t d,
+                               sta_dim3 grid, sta_dim3 tile, bool to_tiled, void* stream) {
+  if (batch < 0 || heads < 0) return STA_ERR_ARG;
+  const int64_t bh = static_cast<int64_t>(batch) * heads;
+  Geometry g;
+  sta_status s = validate_tensor_args(src, dst, bh, d, grid, tile, &g);
+  if (s != STA_OK) return s;
+  if ((s = check_device(nullptr)) != STA_OK) return s;
+  if (bh == 0) return STA_OK;
+  cudaError_t e = launch_reorder(src, dst, bh, d, g, to_tiled, static_cast<cudaStream_t>(stream), heads);
+  return e == cudaSuccess ? STA_OK : cuda_fail(e);
+}
+}  // namespace
+
+sta_status sta_tile_reorder_tokens(const void* src, void* dst, int32_t batch, int32_t heads, int32_t d,
+                                   sta_dim3 grid, sta_dim3 tile, void* stream) {
+  return reorder_tokens_impl(src, dst, batch, heads, d, grid, tile, true, stream);
+}
+
+sta_status sta_tile_unorder_tokens(const void* src, void* dst, int32_t batch, int32_t heads, int32_t d,
+                                   sta_dim3 grid, sta_dim3 tile, void* stream) {
+  return reorder_tokens_impl(src, dst, batch, heads, d, grid, tile, false, stream);
+}
+
+namespace {
 // sta_attention_fwd and sta_attention_fwd_lse: validation, schedule, launch.
 sta_status attention_fwd_impl(const void* q, const void* k, const void* v, void* out, float* lse, int32_t batch,
                               int32_t heads, int32_t d, sta_dim3 grid, sta_dim3 tile,

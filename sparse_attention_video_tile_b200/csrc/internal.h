@@ -87,8 +87,11 @@ inline int32_t window_start_1d(int32_t a, int32_t weff, int32_t n) {
 }
 
 // Kernel launchers (reorder.cu, attention.cu).
+// token_major_heads > 0: the raster side is [B, L, heads, d] with that many
+// heads (batch_heads must then be B * heads); 0: it is [B * heads, L, d].
 cudaError_t launch_reorder(const void* src, void* dst, int64_t batch_heads, int32_t d,
-                           const Geometry& g, bool to_tiled, cudaStream_t stream);
+                           const Geometry& g, bool to_tiled, cudaStream_t stream,
+                           int32_t token_major_heads = 0);
 
 struct DeviceSchedule {
   const WorkItem* items;

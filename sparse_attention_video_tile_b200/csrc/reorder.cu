@@ -7,6 +7,13 @@
 // contiguous in both orders, so each run is one contiguous block of tw*d*2
 // bytes on both sides.  A warp copies a run with 16-byte vector loads and
 // stores; index arithmetic happens once per run, not per element.
+//
+// Token-major variant: the raster side is [B, L, heads, d], the layout of a
+// [B, L, heads * d] projection in a video transformer, and the tiled side is
+// [B, heads, L, d].  A run is then tw token rows heads * d elements apart on
+// the raster side, still one contiguous block on the tiled side; runs of the
+// same tile row and neighbouring heads go to neighbouring warps, so together
+// they read or write the raster rows whole.
 #include <cuda_runtime.h>
 
 #include "internal.h"
@@ -23,6 +30,7 @@ struct RunGeo {
   int32_t H, W;
   int32_t ntile;
   int64_t L;
+  int32_t heads;           // token-major only
 };
 
 __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
@@ -33,7 +41,9 @@ __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
   return r;
 }
 
-template <int CPR>  // 16-byte chunks per token row (d * 2 / 16)
+// CPR: 16-byte chunks per token row (d * 2 / 16).  kTokenMajor: the raster
+// side is [B, L, heads, d] instead of [B, heads, L, d].
+template <int CPR, bool kTokenMajor>
 __global__ void __launch_bounds__(256) reorder_kernel(const uint4* __restrict__ src,
                                                       uint4* __restrict__ dst, RunGeo g,
                                                       int to_tiled) {
@@ -42,8 +52,18 @@ __global__ void __launch_bounds__(256) reorder_kernel(const uint4* __restrict__ 
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
   const int chunks = g.tw * CPR;
   for (int64_t r = warp0; r < g.n_runs; r += nwarps) {
-    const int64_t bh = r / g.runs_per_bh;
-    const int32_t rr = static_cast<int32_t>(r - bh * g.runs_per_bh);
+    int64_t bh, b = 0;
+    int32_t rr, head = 0;
+    if (kTokenMajor) {  // run index = (b * runs_per_bh + rr) * heads + head
+      const int64_t br = r / g.heads;
+      head = static_cast<int32_t>(r - br * g.heads);
+      b = br / g.runs_per_bh;
+      rr = static_cast<int32_t>(br - b * g.runs_per_bh);
+      bh = b * g.heads + head;
+    } else {            // run index = bh * runs_per_bh + rr
+      bh = r / g.runs_per_bh;
+      rr = static_cast<int32_t>(r - bh * g.runs_per_bh);
+    }
     const int32_t tile_id = rr / g.runs_per_tile;
     const int32_t rem = rr - tile_id * g.runs_per_tile;
     const int32_t lt = rem / g.th;
@@ -52,8 +72,10 @@ __global__ void __launch_bounds__(256) reorder_kernel(const uint4* __restrict__ 
     const int32_t ah = (tile_id / g.nW) % g.nH;
     const int32_t aw = tile_id % g.nW;
     const int64_t tiled_row = bh * g.L + static_cast<int64_t>(tile_id) * g.ntile + (lt * g.th + lh) * g.tw;
-    const int64_t raster_row =
-        bh * g.L + (static_cast<int64_t>(at * g.tt + lt) * g.H + (ah * g.th + lh)) * g.W + aw * g.tw;
+    const int64_t n0 = (static_cast<int64_t>(at * g.tt + lt) * g.H + (ah * g.th + lh)) * g.W + aw * g.tw;
+    // raster side: token row j of the run starts at (raster_row + j * rstride) * CPR
+    const int64_t raster_row = kTokenMajor ? (b * g.L + n0) * g.heads + head : bh * g.L + n0;
+    const int64_t rstride = kTokenMajor ? g.heads : 1;
     const uint4* s = src + (to_tiled ? raster_row : tiled_row) * CPR;
     uint4* d = dst + (to_tiled ? tiled_row : raster_row) * CPR;
     for (int base = 0; base < chunks; base += 4 * 32) {
@@ -61,12 +83,14 @@ __global__ void __launch_bounds__(256) reorder_kernel(const uint4* __restrict__ 
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int i = base + u * 32 + lane;
-        if (i < chunks) buf[u] = ld_stream(s + i);
+        const int64_t ri = (i / CPR) * rstride * CPR + (i % CPR);
+        if (i < chunks) buf[u] = ld_stream(s + (to_tiled ? ri : i));
       }
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int i = base + u * 32 + lane;
-        if (i < chunks) d[i] = buf[u];
+        const int64_t ri = (i / CPR) * rstride * CPR + (i % CPR);
+        if (i < chunks) d[to_tiled ? i : ri] = buf[u];
       }
     }
   }
@@ -75,8 +99,9 @@ __global__ void __launch_bounds__(256) reorder_kernel(const uint4* __restrict__ 
 }  // namespace
 
 cudaError_t launch_reorder(const void* src, void* dst, int64_t batch_heads, int32_t d,
-                           const Geometry& geo, bool to_tiled, cudaStream_t stream) {
+                           const Geometry& geo, bool to_tiled, cudaStream_t stream, int32_t token_major_heads) {
   RunGeo g;
+  g.heads = token_major_heads;
   g.runs_per_bh = static_cast<int32_t>(geo.L / geo.tw);
   g.n_runs = batch_heads * g.runs_per_bh;
   g.runs_per_tile = geo.tt * geo.th;
@@ -99,10 +124,15 @@ cudaError_t launch_reorder(const void* src, void* dst, int64_t batch_heads, int3
   if (blocks > max_blocks) blocks = max_blocks;
   const uint4* s = static_cast<const uint4*>(src);
   uint4* dd = static_cast<uint4*>(dst);
-  if (d == 128)
-    reorder_kernel<16><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(s, dd, g, to_tiled ? 1 : 0);
-  else
-    reorder_kernel<8><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(s, dd, g, to_tiled ? 1 : 0);
+  const unsigned nb = static_cast<unsigned>(blocks);
+  const int tt = to_tiled ? 1 : 0;
+  if (token_major_heads > 0) {
+    if (d == 128) reorder_kernel<16, true><<<nb, threads, 0, stream>>>(s, dd, g, tt);
+    else reorder_kernel<8, true><<<nb, threads, 0, stream>>>(s, dd, g, tt);
+  } else {
+    if (d == 128) reorder_kernel<16, false><<<nb, threads, 0, stream>>>(s, dd, g, tt);
+    else reorder_kernel<8, false><<<nb, threads, 0, stream>>>(s, dd, g, tt);
+  }
   return cudaGetLastError();
 }
 

@@ -94,6 +94,25 @@ def test_validation_codes(lib):
     assert lib.sta_attended_pairs(1, 1, sta._d3((4, 8, 8)), sta._d3((3, 4, 4)), sta._windows([(1, 1, 1)])) == -1
 
 
+def _call_tokens(lib, src, dst, batch=1, heads=2, d=128, grid=(4, 8, 8), tile=(2, 4, 4), unorder=False):
+    fn = lib.sta_tile_unorder_tokens if unorder else lib.sta_tile_reorder_tokens
+    return fn(src, dst, batch, heads, d, sta._d3(grid), sta._d3(tile), None)
+
+
+def test_token_major_reorder_validation_codes(lib):
+    # fake pointers, never dereferenced; one tensor is 2 x 256 x 128 bf16 = 128 KB
+    A, B = 0x100000, 0x200000
+    for unorder in (False, True):
+        assert _call_tokens(lib, None, B, unorder=unorder) == 1
+        assert _call_tokens(lib, A, 0, unorder=unorder) == 1
+        assert _call_tokens(lib, A + 8, B, unorder=unorder) == 2
+        assert _call_tokens(lib, A, A + 64 * 1024, unorder=unorder) == 3      # the second half of src
+        assert _call_tokens(lib, A, B, grid=(4, 8, 9), unorder=unorder) == 4
+        assert _call_tokens(lib, A, B, d=32, unorder=unorder) == 6
+        assert _call_tokens(lib, A, B, batch=-1, unorder=unorder) == 10
+        assert _call_tokens(lib, A, B, heads=-2, unorder=unorder) == 10
+
+
 def _call_bwd(lib, base=0x1000000, lse=0x9000000, batch=1, heads=1, d=128, grid=(6, 8, 16), tile=(6, 8, 8),
               windows=((1, 1, 1),), scale=0.1, **ptrs):
     # q, k, v, out, dout, dq, dk, dv spaced 1 MB apart (each [1, 1, 768, 128] bf16 = 192 KB)
@@ -127,8 +146,28 @@ def test_no_cpu_fallback_without_gpu(lib):
         pytest.skip("a GPU is present")
     # valid arguments: the library must report a CUDA/architecture error, not compute on the host
     assert _call_reorder(lib, 0x100000, 0x200000) in (7, 8)
+    assert _call_tokens(lib, 0x100000, 0x200000) in (7, 8)
+    assert _call_tokens(lib, 0x100000, 0x200000, unorder=True) in (7, 8)
+    # the overlap check covers batch * heads * L * d elements: disjoint when that is smaller
+    assert _call_tokens(lib, 0x100000, 0x100000 + 64 * 1024, heads=1) in (7, 8)
     assert _call_attn(lib) in (7, 8)
     assert _call_bwd(lib) in (7, 8)
+
+
+def test_python_paths_refuse_cpu_tensors(lib):
+    """The binding hands device pointers to the library and nothing else: host
+    tensors are refused before any call, on every path."""
+    import torch
+    from sparse_attention_video_tile_b200.autograd import sta_attention
+    cfg = W.custom_config("cpu_refusal", 1, 2, 64, (2, 8, 16), (2, 8, 8), [(1, 1, 1), (1, 1, 2)])
+    q, k, v = W.make_qkv(cfg, 0)
+    tq = q.transpose(1, 2).contiguous()
+    with pytest.raises(ValueError, match="CUDA"):
+        sta.sta_forward_tokens(tq, tq, tq, cfg.grid, cfg.tile, cfg.windows)
+    with pytest.raises(ValueError, match="CUDA"):
+        sta_attention(q, k, v, cfg.grid, cfg.tile, cfg.windows)
+    with pytest.raises(ValueError, match="does not match"):
+        sta.sta_tile_reorder_tokens(tq, torch.empty_like(tq), cfg.grid, cfg.tile)
 
 
 SCHEDULE_CASES = [

@@ -107,3 +107,50 @@ def test_backward_hunyuan_sampled_dq_and_sums():
         dv_sum, do_sum = got[2][0, h].sum(axis=0), do64.sum(axis=0)
         assert np.abs(dv_sum - do_sum).max() <= 1e-2 * np.abs(do_sum).max() + 0.5
         assert np.abs(got[1][0, h].sum(axis=0)).max() <= 1e-2 * np.abs(got[1][0, h]).sum(axis=0).max() + 0.5
+
+
+# ------------------------------------------------------------------ autograd wrapper
+
+AUTOGRAD_CFG = W.custom_config("autograd", 1, 2, 64, (4, 16, 16), (2, 8, 8), [(1, 1, 1), (2, 2, 1)])
+
+
+def test_autograd_matches_oracle_and_explicit_calls():
+    """sta_attention's forward and gradients: the same values as the explicit C-ABI
+    calls (bit for bit) and as the oracle (within the tolerances above)."""
+    from sparse_attention_video_tile_b200.autograd import sta_attention
+    cfg = AUTOGRAD_CFG
+    (q, k, v, do), want_explicit = _gpu_backward(cfg, 3)
+    leaves = [x.cuda().requires_grad_(True) for x in (q, k, v)]
+    out = sta_attention(*leaves, cfg.grid, cfg.tile, cfg.windows, cfg.scale)
+    out.backward(do.cuda())
+    torch.cuda.synchronize()
+    assert sta.sta_check_device_status() == sta.STA_OK
+    want_out = sta.sta_forward(q.cuda(), k.cuda(), v.cuda(), cfg.grid, cfg.tile, cfg.windows, cfg.scale,
+                               fused=False)
+    assert torch.equal(out.detach(), want_out)
+    got = [x.grad.float().cpu().numpy().astype(np.float64) for x in leaves]
+    for name, g, e in zip(("dq", "dk", "dv"), got, want_explicit):
+        assert np.array_equal(g, e), f"{name}: autograd differs from the explicit calls"
+    for h in range(cfg.heads):
+        want = O.sta_attention_backward_head(*(x[0, h].double().numpy() for x in (q, k, v, do)),
+                                             cfg.grid, cfg.tile, cfg.windows[h], cfg.scale)
+        for name, g, w in zip(("dq", "dk", "dv"), got, want):
+            _compare(g[0, h], w, f"autograd head {h} {name}")
+
+
+def test_autograd_token_major_equals_head_major():
+    from sparse_attention_video_tile_b200.autograd import sta_attention
+    cfg = AUTOGRAD_CFG
+    q, k, v = (x.cuda() for x in W.make_qkv(cfg, 4))
+    do = W.make_qkv(cfg, 5)[0].cuda()
+    a = [x.clone().requires_grad_(True) for x in (q, k, v)]
+    b = [x.transpose(1, 2).contiguous().requires_grad_(True) for x in (q, k, v)]
+    out_a = sta_attention(*a, cfg.grid, cfg.tile, cfg.windows, cfg.scale)
+    out_b = sta_attention(*b, cfg.grid, cfg.tile, cfg.windows, cfg.scale, token_major=True)
+    out_a.backward(do)
+    out_b.backward(do.transpose(1, 2))     # a non-contiguous gradient: the wrapper makes it contiguous
+    torch.cuda.synchronize()
+    assert sta.sta_check_device_status() == sta.STA_OK
+    assert torch.equal(out_b.detach().transpose(1, 2), out_a.detach())
+    for x, y in zip(a, b):
+        assert torch.equal(y.grad.transpose(1, 2), x.grad)

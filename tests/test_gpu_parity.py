@@ -80,6 +80,41 @@ def test_reorder_unorder_bit_exact(name):
     torch.cuda.synchronize()
 
 
+@pytest.mark.parametrize("name", ["tiny", "small", "image2d", "hunyuan"])
+def test_token_major_reorder_bit_exact(name):
+    """[B, L, heads, d] raster <-> [B, heads, L, d] tiled, against indexing with the
+    oracle's tile map."""
+    cfg = W.CONFIGS[name]
+    g = torch.Generator(device="cuda").manual_seed(2)
+    x = torch.randn((cfg.batch, cfg.L, cfg.heads, cfg.d), device="cuda", generator=g).to(torch.bfloat16)
+    y = torch.empty((cfg.batch, cfg.heads, cfg.L, cfg.d), device="cuda", dtype=torch.bfloat16)
+    sta.sta_tile_reorder_tokens(x, y, cfg.grid, cfg.tile)
+    m = torch.from_numpy(O.tiled_of_raster(cfg.grid, cfg.tile)).cuda()
+    want = torch.empty_like(y)
+    want[:, :, m, :] = x.transpose(1, 2)
+    assert torch.equal(y, want)
+    del want
+    z = torch.full_like(x, float("nan"))
+    sta.sta_tile_unorder_tokens(y, z, cfg.grid, cfg.tile)
+    assert torch.equal(z, x)
+    torch.cuda.synchronize()
+
+
+@pytest.mark.parametrize("name", ["tiny", "small"])
+def test_forward_tokens_equals_forward(name):
+    """The token-major forward is the head-major forward with both transposes
+    folded into the reorders: equal bit for bit."""
+    cfg = W.CONFIGS[name]
+    q, k, v = (x.cuda() for x in W.make_qkv(cfg, 0))
+    want = sta.sta_forward(q, k, v, cfg.grid, cfg.tile, cfg.windows, cfg.scale, fused=False)
+    tq, tk, tv = (x.transpose(1, 2).contiguous() for x in (q, k, v))
+    got = sta.sta_forward_tokens(tq, tk, tv, cfg.grid, cfg.tile, cfg.windows, cfg.scale)
+    torch.cuda.synchronize()
+    assert sta.sta_check_device_status() == sta.STA_OK
+    assert got.shape == tq.shape
+    assert torch.equal(got.transpose(1, 2), want)
+
+
 # ------------------------------------------------------------------ attention, full outputs
 
 
