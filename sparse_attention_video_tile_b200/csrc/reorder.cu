@@ -44,7 +44,7 @@ __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
 // CPR: 16-byte chunks per token row (d * 2 / 16).  kTokenMajor: the raster
 // side is [B, L, heads, d] instead of [B, heads, L, d].
 template <int CPR, bool kTokenMajor>
-__global__ void __launch_bounds__(256) reorder_kernel(const uint4* __restrict__ src,
+__global__ void __launch_bounds__(256, 6) reorder_kernel(const uint4* __restrict__ src,
                                                       uint4* __restrict__ dst, RunGeo g,
                                                       int to_tiled) {
   const int lane = threadIdx.x & 31;
