@@ -17,8 +17,10 @@ What STA computes, as the sources state it:
     has its own window size.
   * Same paper, review reply on input resolution: the tile is (6, 8, 8) and
     the latent dimensions must be multiples of the tile.
-  * The window rule of the benchmark spec: a window of (wt, wh, ww) tiles
-    around the query tile, its centre clamped so it stays inside the tile grid.
+  * The window rule, for which the pages print no formula: a window of
+    (wt, wh, ww) tiles around the query tile, its centre clamped so that it
+    stays inside the tile grid (the plainest reading of a window that slides
+    tile by tile over a bounded grid).
 
 STA is exact softmax attention under a mask, so this oracle is the masked
 definition written out in fp64 over raster-order tokens: no tiles are
