@@ -1,7 +1,8 @@
-"""Host logic of the head-sharded forward (sparse_attention_video_tile_b200.sharded)
-on CPU: the head partition, and the all-gather of per-rank head slices with two
-gloo ranks.  The attention itself runs only on the GPU (GPU tests); here each rank
-fills its slice with values that identify (batch, head, row, column)."""
+"""Host logic of the sharded forwards (sparse_attention_video_tile_b200.sharded)
+on CPU: the head and token partitions, the all-gather of per-rank head slices,
+and the two all-to-alls of the sequence-sharded forward, with gloo ranks.  The
+attention itself runs only on the GPU (GPU tests); here each rank fills its
+slice with values that identify (batch, head, row, column)."""
 import os
 import socket
 
@@ -10,7 +11,8 @@ import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
 
-from sparse_attention_video_tile_b200.sharded import gather_heads, head_counts, head_range
+from sparse_attention_video_tile_b200.sharded import (gather_heads, head_counts, head_range, heads_to_seq,
+                                                     seq_to_heads, token_range)
 
 
 @pytest.mark.parametrize("heads,world", [(24, 1), (24, 2), (24, 8), (7, 3), (3, 4), (0, 2), (25, 8)])
@@ -58,6 +60,63 @@ def test_gather_reassembles_every_rank_full_output(heads):
         mp.start_processes(_rank_main, args=(world, _free_port(), heads, results), nprocs=world, join=True,
                            start_method="spawn")
         assert dict(results) == {0: True, 1: True}
+
+
+def _a2a_main(rank, world, port, heads, L, results):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        B, d = 2, 4
+        full = _full_reference(B, heads, L, d).transpose(1, 2).contiguous()     # token-major [B, L, heads, d]
+        t0, t1 = token_range(L, world, rank)
+        h0, h1 = head_range(heads, world, rank)
+        local = full[:, t0:t1].contiguous()
+        twice = 2 * local
+        got_q, got_k = seq_to_heads([local, twice], heads, L)                  # one collective for both
+        ok = torch.equal(got_q, full[:, :, h0:h1]) and torch.equal(got_k, 2 * full[:, :, h0:h1])
+        ok = ok and got_q.is_contiguous() and got_k.is_contiguous()
+        # a per-head stand-in for attention, then back to this rank's tokens
+        head_ids = torch.arange(h0, h1, dtype=torch.float32).view(1, 1, -1, 1)
+        back = heads_to_seq(got_q * (head_ids + 1), heads, L)
+        want = local * (torch.arange(heads, dtype=torch.float32).view(1, 1, -1, 1) + 1)
+        results[rank] = bool(ok and torch.equal(back, want))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("heads,L,world", [(24, 64, 2), (5, 7, 2), (1, 9, 2), (4, 10, 3)])
+def test_sequence_shards_exchange_to_head_shards_and_back(heads, L, world):
+    """Uneven token and head splits, and a rank with no heads (1 head, 2 ranks)."""
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as mgr:
+        results = mgr.dict()
+        mp.start_processes(_a2a_main, args=(world, _free_port(), heads, L, results), nprocs=world, join=True,
+                           start_method="spawn")
+        assert dict(results) == {r: True for r in range(world)}
+
+
+def test_token_ranges_partition_the_tokens():
+    for L, world in ((115200, 8), (7, 3), (2, 4)):
+        ranges = [token_range(L, world, r) for r in range(world)]
+        assert ranges[0][0] == 0 and ranges[-1][1] == L
+        assert all(a[1] == b[0] for a, b in zip(ranges, ranges[1:]))
+
+
+@pytest.mark.gpu
+def test_sequence_sharded_single_rank_equals_token_major_forward():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import workloads as W
+    import sparse_attention_video_tile_b200 as sta
+    from sparse_attention_video_tile_b200.build import build
+    from sparse_attention_video_tile_b200.sharded import sta_forward_sequence_sharded
+    build()
+    cfg = W.custom_config("seq_shard", 1, 3, 128, (12, 24, 40), (6, 8, 8), [(1, 3, 3), (3, 3, 3), (1, 1, 1)])
+    q, k, v = (x.cuda().transpose(1, 2).contiguous() for x in W.make_qkv(cfg, 10))
+    want = sta.sta_forward_tokens(q, k, v, cfg.grid, cfg.tile, cfg.windows, cfg.scale)
+    got = sta_forward_sequence_sharded(q, k, v, cfg.grid, cfg.tile, cfg.windows, cfg.scale)
+    torch.cuda.synchronize()
+    assert torch.equal(got, want)
 
 
 @pytest.mark.gpu
