@@ -19,14 +19,23 @@
 //     the per-block operands (K and V, or Q and dO, plus lse and D of the query
 //     block) through a two-stage shared-memory ring with TMA;
 //   * warp 9 issues the tcgen05 MMAs from one thread: S and dP (both operands in
-//     shared memory, fp32 in TMEM), then after the elementwise step the
+//     shared memory, fp32 in TMEM, S in columns 0-127 and dP in 128-255), and the
 //     accumulations with the bf16 P and dS read from TMEM (dQ += dS K, or
-//     dV += P^T dO and dK += dS^T Q);
-//   * warps 0-7 turn S and dP into P and dS: TMEM lane = row, warps w and w+4
-//     take columns 0-63 and 64-127 of the rows of lane quadrant w, and each writes
-//     its P and dS back to TMEM as bf16 over the first 32 of its own columns of S
-//     and dP (so neither overwrites columns the other still reads).  At the end of
-//     an item each warp scales and stores its half of the accumulators' columns.
+//     dV += P^T dO and dK += dS^T Q; accumulators in columns 256-511);
+//   * warps 0-7 do the elementwise step in two phases: TMEM lane = row, warps w
+//     and w+4 take columns 0-63 and 64-127 of the rows of lane quadrant w.  Phase
+//     A turns S into P (fp32, in registers; for dK, dV also stored as bf16 P^T over
+//     S) and releases the S columns; phase B turns dP into dS and stores it as bf16
+//     over dP.  Each warp writes over the first 32 of its own 64 columns, so it never
+//     overwrites columns the other warp still reads.  At the end of an item each
+//     warp scales and stores its half of the accumulators' columns.
+//
+// The two phases let the tensor core run beside the elementwise step: the issuer
+// starts the next block's S as soon as phase A has released the S columns, and the
+// accumulation and the next block's dP as soon as phase B has stored dS, so per
+// block the S product overlaps phase B and the accumulation plus dP overlap the
+// next block's phase A.  Two MMAs that touch the same TMEM columns (the next S over
+// P^T, the next dP over dS) come from the same thread and execute in issue order.
 //
 // Tiles must be multiples of 128 rows, so every block pair in a schedule is fully
 // attended and no mask exists.  Every wait is bounded (see ptx.cuh).
@@ -79,8 +88,10 @@ struct BwdSmem {
   static constexpr int kFixEmpty = kFixFull + 8;
   static constexpr int kKvFull = kFixEmpty + 8;    // [2]
   static constexpr int kKvEmpty = kKvFull + 16;    // [2]
-  static constexpr int kSFull = kKvEmpty + 16;
-  static constexpr int kPFull = kSFull + 8;
+  static constexpr int kSFull = kKvEmpty + 16;    // S (S^T) of a block in TMEM
+  static constexpr int kDFull = kSFull + 8;       // dP (dP^T) of a block in TMEM
+  static constexpr int kSFree = kDFull + 8;       // phase A done: S read (dQ), P^T stored (dK, dV)
+  static constexpr int kPFull = kSFree + 8;       // phase B done: dS (dS^T) stored over dP
   static constexpr int kOFull = kPFull + 8;
   static constexpr int kDrain = kOFull + 8;
   static constexpr int kTmemSlot = kDrain + 8;
@@ -132,7 +143,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(sb + S::kKvEmpty + 8 * s, 1);
     }
     mbar_init(sb + S::kSFull, 1);
-    mbar_init(sb + S::kPFull, 8);   // one arrival per elementwise warp
+    mbar_init(sb + S::kDFull, 1);
+    mbar_init(sb + S::kSFree, 8);   // one arrival per elementwise warp
+    mbar_init(sb + S::kPFull, 8);
     mbar_init(sb + S::kOFull, 1);
     mbar_init(sb + S::kDrain, 1);
     *abort_flag = 0;
@@ -204,63 +217,103 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     __syncwarp();
   } else if (warp == kBwdMma) {
     if (lane == 0) {
+      // Issue order per block b of the CTA's stream (stage b & 1):
+      //   wait phase A of b -> [dK, dV: dV += P^T dO] -> S of b+1 (within an item)
+      //   -> wait phase B of b -> dQ += dS K (or dK += dS^T Q) -> release the stage
+      //   -> [item boundary: wait the next fixed operands, S of b+1] -> dP of b+1.
+      // One thread issues everything, so a later MMA that overwrites an operand an
+      // earlier one reads (S over P^T, dP over dS) executes after it.
       constexpr uint32_t idesc_ss = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t idesc_ts = idesc_bf16_f32(128, D, false, true);
       const uint64_t dfix0 = sdesc_sw128(sb + S::kFix0, 16, 1024);
       const uint64_t dfix1 = sdesc_sw128(sb + S::kFix1, 16, 1024);
       auto koff = [](int k16) -> uint64_t { return static_cast<uint64_t>(((k16 >> 2) * 16384 + (k16 & 3) * 32) >> 4); };
       const uint32_t tS = tmem, tP = tmem + 128, tA0 = tmem + 256, tA1 = tmem + 384;
-      uint32_t seq = 0, blk = 0, nfix = 0;
-      bool ok = true;
-      for (int32_t k = 0; ok; ++k) {
-        const int32_t idx = k * static_cast<int32_t>(gridDim.x) + static_cast<int32_t>(blockIdx.x);
-        if (idx >= p.n_items) break;
-        const int32_t n = p.items[idx].kv_len;
-        ok = mbar_wait(sb + S::kFixFull, nfix & 1, wc, 3);
-        ++nfix;
-        for (int32_t j = 0; j < n && ok; ++j, ++seq, ++blk) {
-          const uint32_t st = seq & 1;
-          ok = mbar_wait(sb + S::kKvFull + 8 * st, (seq >> 1) & 1, wc, 4);
+      auto stage_base = [&](uint32_t b) { return sb + S::kStage0 + (b & 1) * S::kStageBytes; };
+      auto issue_s = [&](uint32_t b) {   // S (S^T) = fix0 str0^T, K-major operands
+        const uint64_t ds0 = sdesc_sw128(stage_base(b), 16, 1024);
+#pragma unroll
+        for (int k16 = 0; k16 < D / 16; ++k16) umma_ss(tS, dfix0 + koff(k16), ds0 + koff(k16), idesc_ss, k16 > 0);
+        umma_commit(sb + S::kSFull);
+      };
+      auto issue_dp = [&](uint32_t b) {  // dP (dP^T) = fix1 str1^T
+        const uint64_t ds1 = sdesc_sw128(stage_base(b) + kBlockBytes, 16, 1024);
+#pragma unroll
+        for (int k16 = 0; k16 < D / 16; ++k16) umma_ss(tP, dfix1 + koff(k16), ds1 + koff(k16), idesc_ss, k16 > 0);
+        umma_commit(sb + S::kDFull);
+      };
+      auto item_len = [&](int32_t kk) -> int32_t {
+        const int32_t idx = kk * static_cast<int32_t>(gridDim.x) + static_cast<int32_t>(blockIdx.x);
+        return idx < p.n_items ? p.items[idx].kv_len : 0;
+      };
+      auto kv_full = [&](uint32_t b) { return mbar_wait(sb + S::kKvFull + 8 * (b & 1), (b >> 1) & 1, wc, 4); };
+      int32_t k = 0, j = 0, n = item_len(0);
+      uint32_t seq = 0, nfix = 0;
+      bool ok = n > 0;
+      if (ok) {
+        ok = mbar_wait(sb + S::kFixFull, 0, wc, 3) && kv_full(0);
+        nfix = 1;
+        if (ok) {
+          tc_fence_after();
+          issue_s(0);
+          issue_dp(0);
+          if (n == 1) umma_commit(sb + S::kFixEmpty);
+        }
+      }
+      while (ok) {
+        const bool new_item = j + 1 == n;               // the next block starts item k + 1
+        const int32_t n_next = new_item ? item_len(k + 1) : n;
+        const bool has_next = n_next > 0;
+        const bool next_is_last = new_item ? n_next == 1 : j + 2 == n;
+        const uint32_t base = stage_base(seq);
+        // accumulations: B operands are the stage's blocks read MN-major (16 rows = 2 KB
+        // per K16 slice); A is bf16 in TMEM, keys (or queries) 0-63 in columns 0-31 and
+        // 64-127 in columns 64-95 of its region
+        const uint64_t dm0 = sdesc_sw128(base, kBlockRows * 128, 1024);
+        const uint64_t dm1 = sdesc_sw128(base + kBlockBytes, kBlockRows * 128, 1024);
+        ok = mbar_wait(sb + S::kSFree, seq & 1, wc, 5);
+        if (!ok) break;
+        tc_fence_after();
+        if (KIND == kDkDv) {
+          // dV += P^T dO (P^T over the S^T columns)
+#pragma unroll
+          for (int k16 = 0; k16 < 8; ++k16)
+            umma_ts(tA0, tS + (k16 >> 2) * 64 + (k16 & 3) * 8, dm1 + static_cast<uint64_t>(k16 * (2048 >> 4)), idesc_ts,
+                    (j > 0 || k16 > 0));
+        }
+        if (has_next && !new_item) {   // next block's S while the elementwise warps finish this one
+          ok = kv_full(seq + 1);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t base = sb + S::kStage0 + st * S::kStageBytes;
-          const uint64_t ds0 = sdesc_sw128(base, 16, 1024), ds1 = sdesc_sw128(base + kBlockBytes, 16, 1024);
-          // S (or S^T) = fix0 str0^T and dP (or dP^T) = fix1 str1^T, both K-major
+          issue_s(seq + 1);
+        }
+        ok = mbar_wait(sb + S::kPFull, seq & 1, wc, 7);
+        if (!ok) break;
+        tc_fence_after();
+        // dQ += dS K, or dK += dS^T Q; dS (dS^T) over the dP (dP^T) columns
 #pragma unroll
-          for (int k16 = 0; k16 < D / 16; ++k16) umma_ss(tS, dfix0 + koff(k16), ds0 + koff(k16), idesc_ss, k16 > 0);
-#pragma unroll
-          for (int k16 = 0; k16 < D / 16; ++k16) umma_ss(tP, dfix1 + koff(k16), ds1 + koff(k16), idesc_ss, k16 > 0);
-          umma_commit(sb + S::kSFull);
-          ok = mbar_wait(sb + S::kPFull, blk & 1, wc, 5);
+        for (int k16 = 0; k16 < 8; ++k16)
+          umma_ts(KIND == kDq ? tA0 : tA1, tP + (k16 >> 2) * 64 + (k16 & 3) * 8,
+                  dm0 + static_cast<uint64_t>(k16 * (2048 >> 4)), idesc_ts, (j > 0 || k16 > 0));
+        umma_commit(sb + S::kKvEmpty + 8 * (seq & 1));
+        if (new_item) umma_commit(sb + S::kOFull);
+        if (!has_next) break;
+        if (new_item) {                 // the next item's fixed operands load after this item's last dP
+          ok = mbar_wait(sb + S::kFixFull, nfix & 1, wc, 3) && kv_full(seq + 1);
+          ++nfix;
           if (!ok) break;
           tc_fence_after();
-          // accumulations: B operands are the streamed blocks read MN-major (rows = K
-          // dimension, 16 rows = 2 KB per slice); A is bf16 in TMEM (8 columns per
-          // slice), keys 0-63 in columns 0-31 and keys 64-127 in columns 64-95
-          const uint64_t dm0 = sdesc_sw128(base, kBlockRows * 128, 1024);
-          const uint64_t dm1 = sdesc_sw128(base + kBlockBytes, kBlockRows * 128, 1024);
-          if (KIND == kDq) {
-            // dQ += dS K
-#pragma unroll
-            for (int k16 = 0; k16 < 8; ++k16)
-              umma_ts(tA0, tS + (k16 >> 2) * 64 + (k16 & 3) * 8, dm0 + static_cast<uint64_t>(k16 * (2048 >> 4)), idesc_ts,
-                      (j > 0 || k16 > 0));
-          } else {
-            // dV += P^T dO, dK += dS^T Q
-#pragma unroll
-            for (int k16 = 0; k16 < 8; ++k16)
-              umma_ts(tA0, tS + (k16 >> 2) * 64 + (k16 & 3) * 8, dm1 + static_cast<uint64_t>(k16 * (2048 >> 4)), idesc_ts,
-                      (j > 0 || k16 > 0));
-#pragma unroll
-            for (int k16 = 0; k16 < 8; ++k16)
-              umma_ts(tA1, tP + (k16 >> 2) * 64 + (k16 & 3) * 8, dm0 + static_cast<uint64_t>(k16 * (2048 >> 4)), idesc_ts,
-                      (j > 0 || k16 > 0));
-          }
-          umma_commit(sb + S::kKvEmpty + 8 * st);
-          if (j + 1 == n) {
-            umma_commit(sb + S::kFixEmpty);
-            umma_commit(sb + S::kOFull);
-          }
+          issue_s(seq + 1);
+        }
+        issue_dp(seq + 1);
+        if (next_is_last) umma_commit(sb + S::kFixEmpty);
+        ++seq;
+        if (new_item) {
+          ++k;
+          j = 0;
+          n = n_next;
+        } else {
+          ++j;
         }
       }
       umma_commit(sb + S::kDrain);
@@ -275,7 +328,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t tS = tl + 64 * hh, tP = tl + 128 + 64 * hh, tA0 = tl + 256, tA1 = tl + 384;
     const float sl2 = p.scale_log2;
     constexpr float kLog2e = 1.4426950408889634f;
-    uint32_t seq = 0, blk = 0;
+    uint32_t seq = 0;
     bool ok = true;
     for (int32_t k = 0; ok; ++k) {
       const int32_t idx = k * static_cast<int32_t>(gridDim.x) + static_cast<int32_t>(blockIdx.x);
@@ -287,9 +340,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         lse2_row = p.lse[grow] * kLog2e;
         d_row = p.dvec[grow];
       }
-      for (int32_t j = 0; j < it.kv_len; ++j, ++seq, ++blk) {
+      for (int32_t j = 0; j < it.kv_len; ++j, ++seq) {
         const uint32_t st = seq & 1;
-        ok = __all_sync(0xffffffffu, mbar_wait(sb + S::kSFull, blk & 1, wc, 7));
+        ok = __all_sync(0xffffffffu, mbar_wait(sb + S::kSFull, seq & 1, wc, 8));
         if (!ok) break;
         if (KIND == kDkDv) {
           // lse and D of the streamed query block, in the stage's shared memory
@@ -297,48 +350,71 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           if (!ok) break;
         }
         tc_fence_after();
-        // lse and D of this warp's 64 columns (dK, dV kernel), read four at a time
         const float4* col_lse4 = reinterpret_cast<const float4*>(smem + S::kStage0 + st * S::kStageBytes +
                                                                  2 * kBlockBytes) + 16 * hh;
         const float4* col_d4 = col_lse4 + 32;
-#pragma unroll 1
-        for (int c = 0; c < 2; ++c) {
-          uint32_t s32[32], p32[32];
-          tmem_ld32(tS + 32 * c, s32);
-          tmem_ld32(tP + 32 * c, p32);
+        // phase A: P (P^T) of this thread's row over this warp's 64 columns, kept in fp32
+        float pf[64];
+        if (KIND == kDq) {
+          uint32_t s_lo[32], s_hi[32];
+          tmem_ld32(tS, s_lo);
+          tmem_ld32(tS + 32, s_hi);
           tmem_wait_ld();
-          uint32_t pk[16], dk[16];
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(sb + S::kSFree);   // S may be overwritten by the next block's
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            pf[i] = ex2_approx(fmaf(__uint_as_float(s_lo[i]), sl2, -lse2_row));
+            pf[32 + i] = ex2_approx(fmaf(__uint_as_float(s_hi[i]), sl2, -lse2_row));
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            uint32_t s32[32], pk[16];
+            tmem_ld32(tS + 32 * c, s32);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+              const float4 lv = col_lse4[8 * c + i / 4];
+              const float l2[4] = {lv.x * kLog2e, lv.y * kLog2e, lv.z * kLog2e, lv.w * kLog2e};
+#pragma unroll
+              for (int u = 0; u < 4; ++u) pf[32 * c + i + u] = ex2_approx(fmaf(__uint_as_float(s32[i + u]), sl2, -l2[u]));
+              pk[i >> 1] = pack_bf16x2(pf[32 * c + i], pf[32 * c + i + 1]);
+              pk[(i >> 1) + 1] = pack_bf16x2(pf[32 * c + i + 2], pf[32 * c + i + 3]);
+            }
+            tmem_st16(tS + 16 * c, pk);   // P^T over the first 32 of this warp's S^T columns
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(sb + S::kSFree);
+        }
+        // phase B: dS = P (dP - D), bf16 over the first 32 of this warp's dP columns
+        ok = __all_sync(0xffffffffu, mbar_wait(sb + S::kDFull, seq & 1, wc, 10));
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t d32[32], dk[16];
+          tmem_ld32(tP + 32 * c, d32);
+          tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < 32; i += 4) {
-            float l2[4], dd[4];
+            float dd[4];
             if (KIND == kDq) {
-#pragma unroll
-              for (int u = 0; u < 4; ++u) {
-                l2[u] = lse2_row;
-                dd[u] = d_row;
-              }
+              dd[0] = dd[1] = dd[2] = dd[3] = d_row;
             } else {
-              const float4 lv = col_lse4[8 * c + i / 4], dv4 = col_d4[8 * c + i / 4];
-              l2[0] = lv.x * kLog2e; l2[1] = lv.y * kLog2e; l2[2] = lv.z * kLog2e; l2[3] = lv.w * kLog2e;
+              const float4 dv4 = col_d4[8 * c + i / 4];
               dd[0] = dv4.x; dd[1] = dv4.y; dd[2] = dv4.z; dd[3] = dv4.w;
             }
-            float pr[4], dsv[4];
+            float dsv[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              pr[u] = ex2_approx(fmaf(__uint_as_float(s32[i + u]), sl2, -l2[u]));
-              dsv[u] = pr[u] * (__uint_as_float(p32[i + u]) - dd[u]);
-            }
-            pk[i >> 1] = pack_bf16x2(pr[0], pr[1]);
-            pk[(i >> 1) + 1] = pack_bf16x2(pr[2], pr[3]);
+            for (int u = 0; u < 4; ++u) dsv[u] = pf[32 * c + i + u] * (__uint_as_float(d32[i + u]) - dd[u]);
             dk[i >> 1] = pack_bf16x2(dsv[0], dsv[1]);
             dk[(i >> 1) + 1] = pack_bf16x2(dsv[2], dsv[3]);
           }
-          if (KIND == kDq) {
-            tmem_st16(tS + 16 * c, dk);    // dS over S
-          } else {
-            tmem_st16(tS + 16 * c, pk);    // P^T over S^T
-            tmem_st16(tP + 16 * c, dk);    // dS^T over dP^T
-          }
+          tmem_st16(tP + 16 * c, dk);
         }
         tmem_wait_st();
         tc_fence_before();
@@ -347,7 +423,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       if (!ok) break;
       // epilogue: the item's accumulators, scaled, as bf16 rows
-      ok = __all_sync(0xffffffffu, mbar_wait(sb + S::kOFull, static_cast<uint32_t>(k) & 1, wc, 8));
+      ok = __all_sync(0xffffffffu, mbar_wait(sb + S::kOFull, static_cast<uint32_t>(k) & 1, wc, 11));
       if (!ok) break;
       tc_fence_after();
       for (int a = 0; a < (KIND == kDq ? 1 : 2); ++a) {
