@@ -179,8 +179,10 @@ sta_status sta_attention_fwd_lse(const void* q, const void* k, const void* v, vo
  * Arithmetic: bf16 operands, fp32 tensor-core accumulation, P and ds rounded to
  * bf16 for the products that take them, bf16 results.
  * The tile must hold a multiple of 128 tokens (for example (6,8,8) or (1,8,16)).
- * The library keeps one fp32 per query row of scratch (grown on demand, freed by
- * sta_shutdown), so the first call of a larger size synchronises the device.
+ * The library keeps one fp32 per query row of scratch (the row terms D; grown on
+ * demand, freed by sta_shutdown), so the first call of a larger size synchronises
+ * the device.  All backward calls on a device share it: calls that overlap on the
+ * GPU (different streams) race on it; order them.
  * Errors: NULL, ALIGN, ALIAS, SHAPE (also: tile not a multiple of 128 tokens),
  * WINDOW, HEADDIM, ARG, ARCH, CUDA.
  */
