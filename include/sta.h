@@ -1,5 +1,7 @@
 /*
- * sta.h - C ABI of the B200 (sm_100a) Sliding Tile Attention forward library.
+ * sta.h - C ABI of the B200 (sm_100a) Sliding Tile Attention library: tile
+ * reorders, the forward pass (with or without its log-sum-exp) and the backward
+ * pass.
  *
  * Method: "Fast Video Generation with Sliding Tile Attention" (arXiv 2502.04507).
  *   - abstract: attention restricted to a local 3D window that moves tile by
@@ -19,7 +21,9 @@
  *
  * Layout conventions (all entry points):
  *   - every q/k/v/out tensor is a contiguous bf16 array [batch, heads, L, d]
- *     (row-major, d fastest), L = T * H * W tokens, d in {64, 128};
+ *     (row-major, d fastest), L = T * H * W tokens, d in {64, 128}; the one
+ *     exception is the raster side of the token-major reorders,
+ *     [batch, L, heads, d];
  *   - raster order: token n = (t * H + h) * W + w;
  *   - tiled order: tiles in raster order over the tile grid, tokens in raster
  *     order inside a tile; tile i occupies rows [i * Ntile, (i + 1) * Ntile).

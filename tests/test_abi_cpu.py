@@ -39,6 +39,33 @@ def test_every_declared_symbol_is_exported(lib):
         assert hasattr(lib, n), n
 
 
+def test_header_is_plain_c_and_matches_the_library(lib, tmp_path):
+    """tests/c/abi_from_c.c binds every entry point to a pointer of its spelled-out
+    type (C99, -Werror), links against libsta.so and calls the host entry points."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("gcc is not installed")
+    pkg = os.path.dirname(sta.LIB_PATH)
+    exe = str(tmp_path / "abi_from_c")
+    cmd = ["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", os.path.join(ROOT, "include"),
+           os.path.join(ROOT, "tests", "c", "abi_from_c.c"), "-o", exe, "-L", pkg, "-l:libsta.so",
+           "-Wl,-rpath," + pkg]
+    subprocess.run(cmd, check=True, capture_output=True, text=True)
+    env = dict(os.environ)
+    import torch   # its bundled CUDA runtime is the one libsta.so resolves at run time
+    env["LD_LIBRARY_PATH"] = os.pathsep.join(
+        [os.path.join(os.path.dirname(torch.__file__), "lib")] +
+        [p for p in (os.path.join(os.path.dirname(os.path.dirname(torch.__file__)), "nvidia", "cuda_runtime", "lib"),)
+         if os.path.isdir(p)] + [env.get("LD_LIBRARY_PATH", "")])
+    out = subprocess.run([exe], check=True, capture_output=True, text=True, env=env).stdout.splitlines()
+    got_map = np.array([int(x) for x in out[0].split()[1:]], dtype=np.int64)
+    assert np.array_equal(got_map, O.tiled_of_raster((4, 8, 8), (2, 4, 4)))
+    assert int(out[1].split()[1]) == O.attended_pairs(1, (4, 8, 8), (2, 4, 4), [(1, 1, 1), (3, 3, 3)])
+    assert out[2].split()[1:] == ["STA_OK", "STA_ERR_SHAPE"]
+    assert out[3].split()[1] == "STA_ERR_NULL"
+
+
 def test_status_strings(lib):
     for code, name in sta.STATUS_NAMES.items():
         assert sta.sta_status_str(code) == name
