@@ -385,7 +385,9 @@ def sta_forward_from_host(q_h, k_h, v_h, out_h, grid, tile, window_per_head, sca
     computation: heads go through in chunks, and while one chunk is computed
     (``sta_forward``) the next is copied in and the previous one copied out, on
     three CUDA streams.  Per head the result equals ``sta_forward`` on device
-    tensors: heads are independent.  Returns once ``out_h`` holds the output."""
+    tensors: heads are independent.  The work starts after what is already queued
+    on the device's current stream (for example a copy that fills the inputs).
+    Returns once ``out_h`` holds the output."""
     import torch
     if q_h.dim() != 4:
         raise ValueError("q must be [batch, heads, L, d]")
@@ -401,8 +403,18 @@ def sta_forward_from_host(q_h, k_h, v_h, out_h, grid, tile, window_per_head, sca
     if heads_per_chunk < 1:
         raise ValueError("heads_per_chunk must be positive")
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(dev):
+        _forward_from_host_chunks(q_h, k_h, v_h, out_h, grid, tile, window_per_head, scale, heads_per_chunk, dev)
+
+
+def _forward_from_host_chunks(q_h, k_h, v_h, out_h, grid, tile, window_per_head, scale, heads_per_chunk, dev):
+    import torch
+    B, Hn = int(q_h.shape[0]), int(q_h.shape[1])
     chunks = [(b, h0, min(Hn, h0 + heads_per_chunk)) for b in range(B) for h0 in range(0, Hn, heads_per_chunk)]
     s_in, s_run, s_out = (torch.cuda.Stream(device=dev) for _ in range(3))
+    caller = torch.cuda.current_stream(dev)
+    for s in (s_in, s_run, s_out):
+        s.wait_stream(caller)
     shape = (1, heads_per_chunk) + tuple(q_h.shape[2:])
     bufs = [[torch.empty(shape, dtype=q_h.dtype, device=dev) for _ in range(3)] for _ in range(2)]
     outs = [None, None]
