@@ -100,6 +100,20 @@ def _stream(stream) -> Optional[int]:
     return stream.cuda_stream
 
 
+def _stream_context(stream):
+    """Makes ``stream`` (None for the current stream, a torch stream or a raw
+    cudaStream_t handle) torch's current stream, so that tensors allocated inside
+    belong to the stream their kernels run on: the caching allocator then reuses
+    their memory only after that stream's work."""
+    import contextlib
+    import torch
+    if stream is None:
+        return contextlib.nullcontext()
+    if isinstance(stream, int):
+        stream = torch.cuda.ExternalStream(stream)
+    return torch.cuda.stream(stream)
+
+
 def _check(status: int, where: str) -> None:
     if status != STA_OK:
         detail = ""
@@ -331,27 +345,29 @@ def sta_forward(q, k, v, grid, tile, window_per_head, scale: Optional[float] = N
       rows, the fused kernel's are 5-D boxes of whole frames).
 
     ``fused=None`` takes the fused call only when the grid is not a tile multiple.
-    Returns the raster-order output.
+    Returns the raster-order output, allocated on ``stream``: use it on another
+    stream only after synchronising with that one.
     """
     import torch
     if scale is None:
         scale = 1.0 / float(q.shape[-1]) ** 0.5
-    out = torch.empty_like(q)
     if fused is None:
         multiple = all(int(a) % int(b) == 0 for a, b in zip(grid, tile))
         fused = not multiple and raster_tile_ok(tile)
-    if fused:
-        sta_attention_fwd_raster(q, k, v, out, grid, tile, window_per_head, scale, stream)
+    with _stream_context(stream):
+        out = torch.empty_like(q)
+        if fused:
+            sta_attention_fwd_raster(q, k, v, out, grid, tile, window_per_head, scale, stream)
+            return out
+        if workspace is None:
+            workspace = tuple(torch.empty_like(q) for _ in range(4))
+        qt, kt, vt, ot = workspace
+        sta_tile_reorder(q, qt, grid, tile, stream)
+        sta_tile_reorder(k, kt, grid, tile, stream)
+        sta_tile_reorder(v, vt, grid, tile, stream)
+        sta_attention_fwd(qt, kt, vt, ot, grid, tile, window_per_head, scale, stream)
+        sta_tile_unorder(ot, out, grid, tile, stream)
         return out
-    if workspace is None:
-        workspace = tuple(torch.empty_like(q) for _ in range(4))
-    qt, kt, vt, ot = workspace
-    sta_tile_reorder(q, qt, grid, tile, stream)
-    sta_tile_reorder(k, kt, grid, tile, stream)
-    sta_tile_reorder(v, vt, grid, tile, stream)
-    sta_attention_fwd(qt, kt, vt, ot, grid, tile, window_per_head, scale, stream)
-    sta_tile_unorder(ot, out, grid, tile, stream)
-    return out
 
 
 def sta_forward_tokens(q, k, v, grid, tile, window_per_head, scale: Optional[float] = None,
@@ -366,16 +382,17 @@ def sta_forward_tokens(q, k, v, grid, tile, window_per_head, scale: Optional[flo
     if scale is None:
         scale = 1.0 / float(q.shape[-1]) ** 0.5
     b, n, h, d = (int(x) for x in q.shape)
-    if workspace is None:
-        workspace = tuple(torch.empty((b, h, n, d), dtype=q.dtype, device=q.device) for _ in range(4))
-    qt, kt, vt, ot = workspace
-    sta_tile_reorder_tokens(q, qt, grid, tile, stream)
-    sta_tile_reorder_tokens(k, kt, grid, tile, stream)
-    sta_tile_reorder_tokens(v, vt, grid, tile, stream)
-    sta_attention_fwd(qt, kt, vt, ot, grid, tile, window_per_head, scale, stream)
-    out = torch.empty_like(q)
-    sta_tile_unorder_tokens(ot, out, grid, tile, stream)
-    return out
+    with _stream_context(stream):
+        if workspace is None:
+            workspace = tuple(torch.empty((b, h, n, d), dtype=q.dtype, device=q.device) for _ in range(4))
+        qt, kt, vt, ot = workspace
+        sta_tile_reorder_tokens(q, qt, grid, tile, stream)
+        sta_tile_reorder_tokens(k, kt, grid, tile, stream)
+        sta_tile_reorder_tokens(v, vt, grid, tile, stream)
+        sta_attention_fwd(qt, kt, vt, ot, grid, tile, window_per_head, scale, stream)
+        out = torch.empty_like(q)
+        sta_tile_unorder_tokens(ot, out, grid, tile, stream)
+        return out
 
 
 def sta_forward_from_host(q_h, k_h, v_h, out_h, grid, tile, window_per_head, scale: Optional[float] = None,

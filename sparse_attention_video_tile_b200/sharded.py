@@ -77,7 +77,7 @@ def sta_forward_head_sharded(q, k, v, grid, tile, window_per_head: Sequence, sca
     (``sta_forward``) and, with ``gather``, the full output is all-gathered.
     Without ``gather`` the rank's slice [B, h1 - h0, L, d] is returned."""
     import torch.distributed as dist
-    from . import sta_forward
+    from . import _stream_context, sta_forward
     heads = int(q.shape[1])
     if len(window_per_head) != heads:
         raise ValueError("one window per head is required")
@@ -87,8 +87,9 @@ def sta_forward_head_sharded(q, k, v, grid, tile, window_per_head: Sequence, sca
     if scale is None:
         scale = 1.0 / float(q.shape[-1]) ** 0.5
     if h1 > h0:
-        local = sta_forward(q[:, h0:h1].contiguous(), k[:, h0:h1].contiguous(), v[:, h0:h1].contiguous(),
-                            grid, tile, list(window_per_head[h0:h1]), scale, stream)
+        with _stream_context(stream):   # the head slices are allocated on the stream that reads them
+            local = sta_forward(q[:, h0:h1].contiguous(), k[:, h0:h1].contiguous(), v[:, h0:h1].contiguous(),
+                                grid, tile, list(window_per_head[h0:h1]), scale, stream)
     else:
         local = q[:, h0:h1].new_empty((q.shape[0], 0) + tuple(q.shape[2:]))
     if not gather or world == 1:
