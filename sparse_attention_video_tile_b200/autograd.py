@@ -15,13 +15,15 @@ Raster tensors are either [B, heads, L, d] (``token_major=False``) or the
 token-major [B, L, heads, d] (``token_major=True``), where the transposes are
 part of the reorders.  The tiled q, k, v, output and log-sum-exp are kept for
 the backward.  Tiles must hold a multiple of 128 tokens and the grid must be a
-tile multiple (the backward kernel's blocking).
+tile multiple (the backward kernel's blocking).  The backward is not itself
+differentiable: a second derivative raises.
 """
 from __future__ import annotations
 
 from typing import Optional, Sequence
 
 import torch
+from torch.autograd.function import once_differentiable
 
 from . import (sta_attention_bwd, sta_attention_fwd_lse, sta_tile_reorder, sta_tile_reorder_tokens,
                sta_tile_unorder, sta_tile_unorder_tokens)
@@ -62,6 +64,7 @@ class STAttentionFunction(torch.autograd.Function):
         return _from_tiled(ot, grid, tile, token_major)
 
     @staticmethod
+    @once_differentiable
     def backward(ctx, dout):
         qt, kt, vt, ot, lse = ctx.saved_tensors
         grid, tile, windows, scale, token_major = ctx.sta_args
