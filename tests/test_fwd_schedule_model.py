@@ -27,8 +27,9 @@ The kernel's current order has two latent hazards, which the model finds:
     V_1 is in it.
 Both need one agent to lag another by a whole block's work, and no GPU run has
 shown either.  The planned order removes both: an O-free barrier (every softmax
-warp arrives after its epilogue reads; the P V issuer waits for it before an
-item's first product) and P_g waited for before V_g.
+thread arrives after its epilogue reads; the P V issuer waits for it before an
+item's first product; modelled per warp, since a warp's threads read O
+together) and P_g waited for before V_g.
 """
 import random
 
