@@ -37,8 +37,13 @@
 //     old reference.  The epilogue adds the two warps' sums, divides and writes
 //     bf16 rows, each warp half of the head dimension.
 //
-// Every barrier that is waited on with a parity can never run two phases ahead
-// of its waiter (the per-buffer S, P and P*V barriers, the Q pair, the ring).
+// Barriers waited on with a parity are meant never to run two phases ahead of
+// their waiter (the per-buffer S, P and P*V barriers, the Q pair, the ring).  Two
+// orderings are not enforced yet: the P*V issuer waits for V_1 (ring load 5, the
+// stage of K_1) before P_1, so that wait could pass early if K_1 had not landed;
+// and an item's first P*V, which overwrites O, is ordered after the epilogue
+// reads of only one warp of each lane-quadrant pair.  Both need one agent to lag
+// another by a whole block; neither has been observed.
 // With Ntile a multiple of 128 no element mask exists at all.  Otherwise (small
 // tiles, ragged tails) the softmax masks whole key tiles outside the row's
 // window and keys past L; padded latents mask the pad keys of boundary blocks.
