@@ -75,7 +75,8 @@ def sta_forward_head_sharded(q, k, v, grid, tile, window_per_head: Sequence, sca
     """STA forward of raster-order [B, heads, L, d] bf16 CUDA tensors held by every
     rank of `group`: each rank computes its own heads with the CUDA path
     (``sta_forward``) and, with ``gather``, the full output is all-gathered.
-    Without ``gather`` the rank's slice [B, h1 - h0, L, d] is returned."""
+    Without ``gather`` the rank's slice [B, h1 - h0, L, d] is returned.  The work
+    and the result are on ``stream`` (default: the current stream)."""
     import torch.distributed as dist
     from . import _stream_context, sta_forward
     heads = int(q.shape[1])
@@ -86,15 +87,18 @@ def sta_forward_head_sharded(q, k, v, grid, tile, window_per_head: Sequence, sca
     h0, h1 = head_range(heads, world, rank)
     if scale is None:
         scale = 1.0 / float(q.shape[-1]) ** 0.5
-    if h1 > h0:
-        with _stream_context(stream):   # the head slices are allocated on the stream that reads them
+    # Everything runs on `stream`: the head slices are allocated on the stream that reads
+    # them, and the all-gather (which orders itself after torch's current stream) starts
+    # after the local forward.
+    with _stream_context(stream):
+        if h1 > h0:
             local = sta_forward(q[:, h0:h1].contiguous(), k[:, h0:h1].contiguous(), v[:, h0:h1].contiguous(),
                                 grid, tile, list(window_per_head[h0:h1]), scale, stream)
-    else:
-        local = q[:, h0:h1].new_empty((q.shape[0], 0) + tuple(q.shape[2:]))
-    if not gather or world == 1:
-        return local
-    return gather_heads(local, heads, group)
+        else:
+            local = q[:, h0:h1].new_empty((q.shape[0], 0) + tuple(q.shape[2:]))
+        if not gather or world == 1:
+            return local
+        return gather_heads(local, heads, group)
 
 
 def _world_rank(group):
