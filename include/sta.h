@@ -234,8 +234,10 @@ sta_status sta_attention_fwd_raster(const void* q, const void* k, const void* v,
  * overlap on the GPU (different streams) race on the array; order them.
  * The first call on a device looks up the array's device address
  * (cudaGetSymbolAddress); make that first call before any stream capture.
- * Bounded-wait timeouts of this variant are recorded in the scratch status word
- * and are not reported by sta_check_device_status.
+ * Bounded-wait timeouts of this variant are recorded in the array's status word,
+ * which sta_check_device_status reports and clears like the other entry points'
+ * (synchronise the stream the call ran on through it).  After sta_shutdown, or a
+ * device reset, the next call sets the device up again.
  */
 sta_status sta_attention_fwd_noalloc(const void* q, const void* k, const void* v, void* out,
                                      int32_t batch, int32_t heads, int32_t d, sta_dim3 grid,
@@ -243,18 +245,23 @@ sta_status sta_attention_fwd_noalloc(const void* q, const void* k, const void* v
                                      void* stream);
 
 /*
- * Synchronises `stream` and reports whether any kernel of this library gave up
- * on a bounded wait since the last check (STA_ERR_TIMEOUT), then clears the
- * flag.  Returns STA_ERR_CUDA if the stream has a pending CUDA error.
+ * Synchronises `stream` and reports whether any kernel of this library on the
+ * current device gave up on a bounded wait since the last check
+ * (STA_ERR_TIMEOUT), then clears the flag.  The flags read are the allocating
+ * entry points' status word and, once sta_attention_fwd_noalloc has run on the
+ * device, that entry point's own.  Returns STA_ERR_CUDA if the stream has a
+ * pending CUDA error.
  */
 sta_status sta_check_device_status(void* stream);
 
 /*
- * Self-test of the bounded-wait path: launches one block whose threads wait on
+ * Self-test of the bounded-wait path: for each status word of the current
+ * device (see sta_check_device_status) launches one block whose threads wait on
  * a shared-memory barrier that nothing completes, with a limit of `limit_ns`
- * nanoseconds (clamped to [1e5, 5e9]), and synchronises `stream`.  A correct
- * library returns STA_ERR_TIMEOUT and leaves the context usable.  No schedule
- * or tensor is touched.
+ * nanoseconds (clamped to [1e5, 5e9]) and the expiry recorded in that word, then
+ * synchronises `stream`.  Returns STA_ERR_TIMEOUT if every word recorded its
+ * expiry (a correct library), and leaves the words cleared and the context
+ * usable.  No schedule or tensor is touched.
  */
 sta_status sta_selftest_bounded_wait(uint64_t limit_ns, void* stream);
 

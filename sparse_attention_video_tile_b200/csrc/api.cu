@@ -19,11 +19,6 @@ namespace {
 
 thread_local std::string g_last_cuda_error;
 
-sta_status cuda_fail(cudaError_t e) {
-  g_last_cuda_error = cudaGetErrorString(e);
-  return STA_ERR_CUDA;
-}
-
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per bounded wait
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -165,6 +160,12 @@ sta_status validate_tensor_args(const void* src, const void* dst, int64_t batch_
 }
 
 }  // namespace
+
+sta_status cuda_fail(cudaError_t e) {
+  g_last_cuda_error = cudaGetErrorString(e);
+  return STA_ERR_CUDA;
+}
+
 }  // namespace sta
 
 using namespace sta;
@@ -441,22 +442,46 @@ sta_status sta_attention_fwd_raster(const void* q, const void* k, const void* v,
   return e == cudaSuccess ? STA_OK : cuda_fail(e);
 }
 
+namespace {
+// Reads a device status word; if it is set, clears it.  *set tells which.
+sta_status read_and_clear(int32_t* word, bool* set) {
+  int32_t flag = 0;
+  cudaError_t e = cudaMemcpy(&flag, word, sizeof(flag), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e);
+  *set = flag != 0;
+  if (*set && (e = cudaMemset(word, 0, sizeof(int32_t))) != cudaSuccess) return cuda_fail(e);
+  return STA_OK;
+}
+
+// The status words of the current device: the allocating entry points' word (if
+// allocated) and the no-alloc entry point's word (if set up).  Caller holds no lock.
+int status_words(int dev, int32_t* words[2]) {
+  int n = 0;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    auto it = g_devices.find(dev);
+    if (it != g_devices.end() && it->second.d_err) words[n++] = it->second.d_err;
+  }
+  if (int32_t* w = noalloc_status_word(dev)) words[n++] = w;
+  return n;
+}
+}  // namespace
+
 sta_status sta_check_device_status(void* stream) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e);
   if ((e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream))) != cudaSuccess) return cuda_fail(e);
-  std::lock_guard<std::mutex> lock(g_mu);
-  auto it = g_devices.find(dev);
-  if (it == g_devices.end() || !it->second.d_err) return STA_OK;
-  int32_t flag = 0;
-  if ((e = cudaMemcpy(&flag, it->second.d_err, sizeof(flag), cudaMemcpyDeviceToHost)) != cudaSuccess)
-    return cuda_fail(e);
-  if (flag != 0) {
-    if ((e = cudaMemset(it->second.d_err, 0, sizeof(int32_t))) != cudaSuccess) return cuda_fail(e);
-    return STA_ERR_TIMEOUT;
+  int32_t* words[2];
+  const int n = status_words(dev, words);
+  bool any = false;
+  for (int i = 0; i < n; ++i) {
+    bool set = false;
+    sta_status s = read_and_clear(words[i], &set);
+    if (s != STA_OK) return s;
+    any = any || set;
   }
-  return STA_OK;
+  return any ? STA_ERR_TIMEOUT : STA_OK;
 }
 
 sta_status sta_selftest_bounded_wait(uint64_t limit_ns, void* stream) {
@@ -465,16 +490,26 @@ sta_status sta_selftest_bounded_wait(uint64_t limit_ns, void* stream) {
   sta_status s;
   int dev = 0;
   if ((s = check_device(&dev)) != STA_OK) return s;
-  int32_t* err = nullptr;
   {
     std::lock_guard<std::mutex> lock(g_mu);
     DeviceState* st = nullptr;
     if ((s = device_state(dev, &st)) != STA_OK) return s;
-    err = st->d_err;
   }
-  cudaError_t e = launch_selftest_wait(err, limit_ns, static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(e);
-  return sta_check_device_status(stream);
+  // One run-out wait per status word of the device; each word must report it.
+  int32_t* words[2];
+  const int n = status_words(dev, words);
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  for (int i = 0; i < n; ++i)
+    if ((e = launch_selftest_wait(words[i], limit_ns, cs)) != cudaSuccess) return cuda_fail(e);
+  if ((e = cudaStreamSynchronize(cs)) != cudaSuccess) return cuda_fail(e);
+  bool all = n > 0;
+  for (int i = 0; i < n; ++i) {
+    bool set = false;
+    if ((s = read_and_clear(words[i], &set)) != STA_OK) return s;
+    all = all && set;
+  }
+  return all ? STA_ERR_TIMEOUT : STA_OK;
 }
 
 void sta_shutdown(void) {
@@ -492,6 +527,7 @@ void sta_shutdown(void) {
     kv.second.dvec_rows = 0;
   }
   g_devices.clear();
+  noalloc_reset();
   cudaSetDevice(cur);
 }
 

@@ -37,13 +37,8 @@
 //     old reference.  The epilogue adds the two warps' sums, divides and writes
 //     bf16 rows, each warp half of the head dimension.
 //
-// Barriers waited on with a parity are meant never to run two phases ahead of
-// their waiter (the per-buffer S, P and P*V barriers, the Q pair, the ring).  Two
-// orderings are not enforced yet: the P*V issuer waits for V_1 (ring load 5, the
-// stage of K_1) before P_1, so that wait could pass early if K_1 had not landed;
-// and an item's first P*V, which overwrites O, is ordered after the epilogue
-// reads of only one warp of each lane-quadrant pair.  Both need one agent to lag
-// another by a whole block; neither has been observed.
+// Every barrier that is waited on with a parity can never run two phases ahead
+// of its waiter (the per-buffer S, P and P*V barriers, the Q pair, the ring).
 // With Ntile a multiple of 128 no element mask exists at all.  Otherwise (small
 // tiles, ragged tails) the softmax masks whole key tiles outside the row's
 // window and keys past L; padded latents mask the pad keys of boundary blocks.
@@ -118,7 +113,8 @@ struct Smem {
   static constexpr int kOut = kPvDone + 8 * kSBufs;        // [lane quadrant]: outcome of each block published
   static constexpr int kLxBar = kOut + 8 * 4;              // [lane quadrant]: half row sums written
   static constexpr int kOFull = kLxBar + 8 * 4;
-  static constexpr int kDrain = kOFull + 8;
+  static constexpr int kOFree = kOFull + 8;                // every softmax warp done reading an item's O
+  static constexpr int kDrain = kOFree + 8;
   static constexpr int kDrainS = kDrain + 8;
   static constexpr int kTmemSlot = kDrainS + 8;
   static constexpr int kAbort = kTmemSlot + 4;
@@ -203,6 +199,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(sb + S::kLxBar + 8 * q, 64);   // every thread of the pair
     }
     mbar_init(sb + S::kOFull, 1);
+    mbar_init(sb + S::kOFree, 256); // one arrival per softmax thread
     mbar_init(sb + S::kDrain, 1);
     mbar_init(sb + S::kDrainS, 1);
     *abort_flag = 0;
@@ -348,7 +345,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int32_t g = c.g;
           const int b = g % kSBufs;
           const uint32_t seq = static_cast<uint32_t>(min(G + g, 2 * g + 3));
-          ok = wait_load(seq, 6) && mbar_wait(sb + S::kPFull + 8 * b, (g / kSBufs) & 1, wc, 5);
+          // P_g first: it implies S_g ran, so K_g (the load before V_g on a ring stage
+          // when g = 1) has landed and the parity wait for V_g cannot pass early.  An
+          // item's first product (accumulate = 0) also waits until every softmax warp
+          // has read the previous item's O.
+          ok = mbar_wait(sb + S::kPFull + 8 * b, (g / kSBufs) & 1, wc, 5) && wait_load(seq, 6) &&
+               (c.j != 0 || c.k == 0 || mbar_wait(sb + S::kOFree, static_cast<uint32_t>(c.k - 1) & 1, wc, 15));
           if (!ok) break;
           tc_fence_after();
           const uint32_t st = seq % kStages;
@@ -647,6 +649,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         tc_fence_before();
+        mbar_arrive(sb + S::kOFree);   // this thread's reads of O are complete
       }
       cur.next(p);
     }

@@ -128,4 +128,18 @@ cudaError_t launch_backward(const void* q, const void* k, const void* v, const v
 
 cudaError_t launch_selftest_wait(int32_t* err_flag, uint64_t limit_ns, cudaStream_t stream);
 
+// Records the text of a failed CUDA call for sta_last_cuda_error and returns
+// STA_ERR_CUDA (api.cu).
+sta_status cuda_fail(cudaError_t e);
+
+// The no-alloc entry point's status word on device `dev` (a device address inside
+// its static scratch array), or null while that entry point has not been set up on
+// the device (noalloc.cu).
+int32_t* noalloc_status_word(int dev);
+
+// Forgets every device's no-alloc set-up (scratch address and uploaded schedule),
+// so that the next call on a device looks the address up and uploads again
+// (noalloc.cu).  Called by sta_shutdown.
+void noalloc_reset();
+
 }  // namespace sta

@@ -22,6 +22,12 @@
 // again whenever the configuration differs from the last one uploaded on the
 // device.  Calls that overlap on the GPU (for instance on two streams) race on
 // the array and must be ordered by the caller.
+//
+// A kernel that gives up on a bounded wait records it in the status word, which
+// sta_check_device_status reads (and clears) beside the allocating entry points'
+// word.  sta_shutdown forgets the set-up, so after it (or after a device reset,
+// which re-initialises the array) the next call looks the address up again and
+// uploads its schedule anew.
 #include <cuda_runtime.h>
 
 #include <array>
@@ -57,6 +63,19 @@ std::array<NoAllocDevice, kMaxDevices> g_noalloc;
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 }  // namespace
+
+int32_t* noalloc_status_word(int dev) {
+  if (dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  const NoAllocDevice& nd = g_noalloc[dev];
+  return nd.ready ? reinterpret_cast<int32_t*>(nd.base) : nullptr;
+}
+
+void noalloc_reset() {
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  for (NoAllocDevice& nd : g_noalloc) nd = NoAllocDevice();
+}
+
 }  // namespace sta
 
 using namespace sta;
@@ -86,11 +105,11 @@ extern "C" sta_status sta_attention_fwd_noalloc(const void* q, const void* k, co
 
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return STA_ERR_CUDA;
+  if (e != cudaSuccess) return cuda_fail(e);
   int major = 0, minor = 0;
-  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
-    return STA_ERR_CUDA;
+  if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
+      (e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess)
+    return cuda_fail(e);
   if (major != 10 || minor != 0) return STA_ERR_ARCH;
   if (dev < 0 || dev >= kMaxDevices) return STA_ERR_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -101,7 +120,8 @@ extern "C" sta_status sta_attention_fwd_noalloc(const void* q, const void* k, co
     // Once per device, with the device current: the scratch array's device address.
     void* ptr = nullptr;
     e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
-    if (e != cudaSuccess || ptr == nullptr) return STA_ERR_CUDA;
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (ptr == nullptr) return cuda_fail(cudaErrorInvalidSymbol);
     nd.base = static_cast<unsigned char*>(ptr);
     nd.ready = true;
   }
@@ -126,13 +146,13 @@ extern "C" sta_status sta_attention_fwd_noalloc(const void* q, const void* k, co
     // earlier work (so a previous call on this stream is done with the array)
     // and returns once the source has been staged.
     nd.has_schedule = false;
-    if (cudaMemcpyAsync(nd.base + off_items, hs.items.data(), hs.items.size() * sizeof(WorkItem),
-                        cudaMemcpyHostToDevice, st) != cudaSuccess ||
-        cudaMemcpyAsync(nd.base + off_kv, hs.kv_rows.data(), hs.kv_rows.size() * sizeof(int32_t),
-                        cudaMemcpyHostToDevice, st) != cudaSuccess ||
-        cudaMemcpyAsync(nd.base + off_win, hs.head_win.data(), hs.head_win.size() * sizeof(int16_t),
-                        cudaMemcpyHostToDevice, st) != cudaSuccess)
-      return STA_ERR_CUDA;
+    if ((e = cudaMemcpyAsync(nd.base + off_items, hs.items.data(), hs.items.size() * sizeof(WorkItem),
+                             cudaMemcpyHostToDevice, st)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(nd.base + off_kv, hs.kv_rows.data(), hs.kv_rows.size() * sizeof(int32_t),
+                             cudaMemcpyHostToDevice, st)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(nd.base + off_win, hs.head_win.data(), hs.head_win.size() * sizeof(int16_t),
+                             cudaMemcpyHostToDevice, st)) != cudaSuccess)
+      return cuda_fail(e);
     nd.sched = std::move(hs);
     nd.key = std::move(key);
     nd.off_items = off_items;
@@ -141,7 +161,7 @@ extern "C" sta_status sta_attention_fwd_noalloc(const void* q, const void* k, co
     nd.has_schedule = true;
   }
   // The status word must start at zero for every call.
-  if (cudaMemsetAsync(nd.base, 0, kStatusBytes, st) != cudaSuccess) return STA_ERR_CUDA;
+  if ((e = cudaMemsetAsync(nd.base, 0, kStatusBytes, st)) != cudaSuccess) return cuda_fail(e);
 
   DeviceSchedule ds{reinterpret_cast<const WorkItem*>(nd.base + nd.off_items),
                     reinterpret_cast<const int32_t*>(nd.base + nd.off_kv),
@@ -149,5 +169,5 @@ extern "C" sta_status sta_attention_fwd_noalloc(const void* q, const void* k, co
                     static_cast<int32_t>(nd.sched.items.size()), nd.sched.masked};
   e = launch_attention(q, k, v, out, batch, heads, d, g, ds, scale, reinterpret_cast<int32_t*>(nd.base),
                        kNoAllocWaitLimitNs, st);
-  return e == cudaSuccess ? STA_OK : STA_ERR_CUDA;
+  return e == cudaSuccess ? STA_OK : cuda_fail(e);
 }

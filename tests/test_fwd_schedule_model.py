@@ -17,19 +17,20 @@ Every read checks that it sees the version it wants (the S or P of its block in
 its quadrant's rows, O accumulated up to the right block, the right stage, Q
 buffer, outcome slot and row-sum slot).
 
-The kernel's current order has two latent hazards, which the model finds:
-  * "O overwritten": the first P V of an item (accumulate = 0) is ordered after
-    the epilogue reads of O only for the warp that publishes the item's next
-    block, not for its partner;
-  * "V stage read": the P V issuer waits for V_1 (ring load 5, stage 1 with
-    four stages) before P_1; if K_1 (ring load 1, same stage) has not landed
-    yet, that parity wait passes at once, and P V_1 may read the stage before
-    V_1 is in it.
-Both need one agent to lag another by a whole block's work, and no GPU run has
-shown either.  The planned order removes both: an O-free barrier (every softmax
-thread arrives after its epilogue reads; the P V issuer waits for it before an
-item's first product; modelled per warp, since a warp's threads read O
-together) and P_g waited for before V_g.
+The kernel enforces two orderings that an earlier version of it lacked, and the
+model shows what each one prevents:
+  * "O overwritten": the first P V of an item (accumulate = 0) must come after
+    the epilogue reads of O by every softmax warp.  Ordering it only after the
+    warp that publishes the item's next block leaves the partner warp of that
+    lane quadrant unprotected.  The kernel has an O-free barrier: every softmax
+    thread arrives after its epilogue reads, and the P V issuer waits for it
+    before an item's first product (modelled per warp, since a warp's threads
+    read O together).
+  * "V stage read": the P V issuer must wait for P_g before V_g.  Waiting for
+    V_1 (ring load 5, stage 1 with four stages) first lets that parity wait
+    pass at once if K_1 (ring load 1, same stage) has not landed yet, and P V_1
+    could then read the stage before V_1 is in it.  P_g implies S_g ran, so K_g
+    (and every earlier load on V_g's stage) has landed.
 """
 import random
 
@@ -281,16 +282,20 @@ def _failures(n, seed, **kw):
     return out
 
 
-def test_planned_order_has_no_deadlock_and_no_stale_read():
+def test_kernel_order_has_no_deadlock_and_no_stale_read():
+    # the order of csrc/attention.cu: O-free barrier, P_g before V_g
     assert _failures(3000, 1, o_free=True, p_before_v=True) == []
 
 
-def test_current_kernel_order_has_exactly_the_two_known_hazards():
+def test_without_the_two_orderings_the_model_finds_both_hazards():
+    # the earlier order (V_g before P_g, no O-free barrier) has exactly these two
     fails = _failures(6000, 2)
     kinds = {f.split(":")[0] for f in fails}
     assert kinds == {O_OVERWRITE, V_STAGE}, kinds
     # the O-free barrier alone leaves only the (rarer) stage hazard
     assert all(f.startswith(V_STAGE) for f in _failures(1500, 3, o_free=True))
+    # P before V alone leaves only the O hazard
+    assert all(f.startswith(O_OVERWRITE) for f in _failures(1500, 5, p_before_v=True))
 
 
 @pytest.mark.parametrize("mutation", ["no_pvdone_wait", "no_outcome_read"])

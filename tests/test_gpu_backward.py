@@ -89,21 +89,59 @@ def test_backward_full_parity(cfg):
                 _compare(g, w, f"{cfg.name} b{b} h{h} {name}")
 
 
-def test_backward_hunyuan_sampled_dq_and_sums():
+def _key_tile_rows(cfg, a):
+    """Raster rows of the tokens of tile a = (at, ah, aw)."""
+    T, H, Wd = cfg.grid
+    tt, th, tw = cfg.tile
+    t, h, w = np.meshgrid(np.arange(a[0] * tt, (a[0] + 1) * tt), np.arange(a[1] * th, (a[1] + 1) * th),
+                          np.arange(a[2] * tw, (a[2] + 1) * tw), indexing="ij")
+    return np.sort(((t * H + h) * Wd + w).ravel())
+
+
+def _dk_dv_of_key_tile(cfg, q64, k64, v64, do64, window, a):
+    """Exact dk, dv of the keys of tile a from the oracle's chain rule.  Only the
+    query rows whose window contains tile a have P != 0 on its keys, so they alone
+    contribute; each takes its softmax over its own window, for which the keys of
+    the union of those windows suffice (the mask removes the rest)."""
+    coords = O.raster_coords(cfg.grid)
+    krows = _key_tile_rows(cfg, a)
+    queries = np.nonzero(O.sta_mask(coords, coords[krows[:1]], cfg.grid, cfg.tile, window)[:, 0])[0]
+    union = np.zeros(cfg.L, dtype=bool)
+    for r0 in range(0, queries.size, 2048):
+        union |= O.sta_mask(coords[queries[r0:r0 + 2048]], coords, cfg.grid, cfg.tile, window).any(axis=0)
+    keys = np.nonzero(union)[0]
+    pos = np.searchsorted(keys, krows)
+    assert np.array_equal(keys[pos], krows)
+    dk = np.zeros((krows.size, k64.shape[1]))
+    dv = np.zeros((krows.size, v64.shape[1]))
+    for r0 in range(0, queries.size, 512):
+        sel = queries[r0:r0 + 512]
+        mask = O.sta_mask(coords[sel], coords[keys], cfg.grid, cfg.tile, window)
+        _, gk, gv = O.masked_softmax_attention_backward(q64[sel], k64[keys], v64[keys], mask, cfg.scale, do64[sel])
+        dk += gk[pos]
+        dv += gv[pos]
+    return krows, dk, dv
+
+
+def test_backward_hunyuan_full_size_dq_rows_and_dk_dv_tiles():
     """At the full 30x48x80 size: dq of sampled rows (a row's dq needs only its own
-    window), and for dk and dv the closed forms sum_k dv = sum_q dO and
-    sum_k dk = 0, which hold at any size."""
+    window), dk and dv element by element on one whole key tile per head (an
+    interior tile and a corner tile), and the closed forms sum_k dv = sum_q dO and
+    sum_k dk = 0 over all keys."""
     cfg = W.CONFIGS["hunyuan"]
-    heads = (0, 13)
+    cases = ((0, (2, 3, 5)), (13, (0, 0, 0)))
     (q, k, v, do), got = _gpu_backward(cfg, seed=7)
     rng = np.random.default_rng(3)
     coords = O.raster_coords(cfg.grid)
-    for h in heads:
+    for h, a in cases:
         rows = np.sort(rng.choice(cfg.L, 48, replace=False))
         q64, k64, v64, do64 = (x[0, h].double().numpy() for x in (q, k, v, do))
         mask = O.sta_mask(coords[rows], coords, cfg.grid, cfg.tile, cfg.windows[h])
         want_dq, _, _ = O.masked_softmax_attention_backward(q64[rows], k64, v64, mask, cfg.scale, do64[rows])
         _compare(got[0][0, h][rows], want_dq, f"hunyuan h{h} dq rows")
+        krows, want_dk, want_dv = _dk_dv_of_key_tile(cfg, q64, k64, v64, do64, cfg.windows[h], a)
+        _compare(got[1][0, h][krows], want_dk, f"hunyuan h{h} dk of tile {a}")
+        _compare(got[2][0, h][krows], want_dv, f"hunyuan h{h} dv of tile {a}")
         dv_sum, do_sum = got[2][0, h].sum(axis=0), do64.sum(axis=0)
         assert np.abs(dv_sum - do_sum).max() <= 1e-2 * np.abs(do_sum).max() + 0.5
         assert np.abs(got[1][0, h].sum(axis=0)).max() <= 1e-2 * np.abs(got[1][0, h]).sum(axis=0).max() + 0.5

@@ -215,6 +215,34 @@ def test_attention_stress_shapes(cfg):
     _full_parity(cfg, seed=3)
 
 
+# Many work items per CTA, every row against the oracle.  18 heads of the small
+# latent give 18 x 90 = 1620 query blocks on a grid of one CTA per SM (about 11
+# items per CTA on 148 SMs).  The mixed windows make items of 3 to 27 key blocks,
+# so item boundaries come often: each one hands O from the epilogue of one item
+# to the first, overwriting P V of the next, and every such hand-over is checked.
+MANY_ITEMS = W.custom_config("many_items", 1, 18, 128, (12, 24, 40), (6, 8, 8),
+                             [(1, 1, 1), (3, 3, 3), (1, 3, 3), (2, 3, 5), (1, 2, 1), (3, 1, 2)] * 3)
+
+
+@pytest.mark.parametrize("fused", [False, True], ids=["three_call", "fused"])
+def test_attention_many_items_per_cta_full_oracle(fused):
+    _full_parity(MANY_ITEMS, seed=21, fused=fused)
+
+
+def test_attention_hunyuan_bitwise_repeatable():
+    """Five full forwards of the HunyuanVideo-shaped workload give the same bits:
+    a race between the pipeline's agents would show up as run-to-run differences."""
+    cfg = W.CONFIGS["hunyuan"]
+    q, k, v = (x.cuda() for x in W.make_qkv(cfg, 3))
+    first = sta.sta_forward(q, k, v, cfg.grid, cfg.tile, cfg.windows, cfg.scale, fused=False)
+    for _ in range(4):
+        again = sta.sta_forward(q, k, v, cfg.grid, cfg.tile, cfg.windows, cfg.scale, fused=False)
+        torch.cuda.synchronize()
+        assert torch.equal(again, first)
+        del again
+    assert sta.sta_check_device_status() == sta.STA_OK
+
+
 # ------------------------------------------------------------------ attention, sampled rows at full size
 
 

@@ -112,11 +112,20 @@ def test_sequence_sharded_single_rank_equals_token_major_forward():
     from sparse_attention_video_tile_b200.sharded import sta_forward_sequence_sharded
     build()
     cfg = W.custom_config("seq_shard", 1, 3, 128, (12, 24, 40), (6, 8, 8), [(1, 3, 3), (3, 3, 3), (1, 1, 1)])
-    q, k, v = (x.cuda().transpose(1, 2).contiguous() for x in W.make_qkv(cfg, 10))
+    import numpy as np
+    import oracle.sta_oracle as O
+    q0, k0, v0 = W.make_qkv(cfg, 10)
+    q, k, v = (x.cuda().transpose(1, 2).contiguous() for x in (q0, k0, v0))
     want = sta.sta_forward_tokens(q, k, v, cfg.grid, cfg.tile, cfg.windows, cfg.scale)
     got = sta_forward_sequence_sharded(q, k, v, cfg.grid, cfg.tile, cfg.windows, cfg.scale)
     torch.cuda.synchronize()
     assert torch.equal(got, want)
+    out = got.float().cpu().numpy().astype(np.float64)        # [B, L, heads, d]
+    for h in range(cfg.heads):
+        ref = O.sta_attention_head(q0[0, h].double().numpy(), k0[0, h].double().numpy(), v0[0, h].double().numpy(),
+                                   cfg.grid, cfg.tile, cfg.windows[h], cfg.scale)
+        assert np.abs(out[0, :, h] - ref).max() <= 1e-2
+        assert np.linalg.norm(out[0, :, h] - ref) / np.linalg.norm(ref) <= 5e-3
 
 
 @pytest.mark.gpu
@@ -142,3 +151,65 @@ def test_head_slices_on_one_gpu_equal_the_full_forward():
     torch.cuda.synchronize()
     assert torch.equal(alone, full)
     assert torch.equal(torch.cat(parts, dim=1), full)
+
+
+def _gpu_rank_main(rank, world, port, results):
+    """One rank of the head-sharded forward on the one GPU of the run: it computes
+    its own heads (no collective: gather=False) and checks them against the oracle."""
+    import numpy as np
+    import oracle.sta_oracle as O
+    import workloads as W
+    import sparse_attention_video_tile_b200 as sta
+    from sparse_attention_video_tile_b200.sharded import sta_forward_head_sharded
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        torch.cuda.set_device(0)
+        sta.load_library()
+        cfg = W.custom_config("shard_oracle", 1, 5, 128, (12, 24, 40), (6, 8, 8),
+                              [(1, 3, 3), (3, 3, 3), (1, 1, 1), (3, 5, 5), (2, 3, 5)])
+        q, k, v = W.make_qkv(cfg, 9)
+        part = sta_forward_head_sharded(q.cuda(), k.cuda(), v.cuda(), cfg.grid, cfg.tile, cfg.windows, cfg.scale,
+                                        gather=False)
+        torch.cuda.synchronize()
+        h0, h1 = head_range(cfg.heads, world, rank)
+        assert part.shape == (1, h1 - h0, cfg.L, cfg.d), part.shape
+        assert sta.sta_check_device_status() == sta.STA_OK
+        got = part.float().cpu().numpy().astype(np.float64)
+        worst = (0.0, 0.0)
+        for i, h in enumerate(range(h0, h1)):
+            want = O.sta_attention_head(q[0, h].double().numpy(), k[0, h].double().numpy(), v[0, h].double().numpy(),
+                                        cfg.grid, cfg.tile, cfg.windows[h], cfg.scale)
+            err = float(np.abs(got[0, i] - want).max())
+            rel = float(np.linalg.norm(got[0, i] - want) / np.linalg.norm(want))
+            worst = (max(worst[0], err), max(worst[1], rel))
+        results[rank] = (h0, h1, worst[0], worst[1])
+    except Exception as e:  # reported to the parent
+        results[rank] = repr(e)
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.gpu
+def test_head_sharded_slices_match_the_oracle():
+    """Each of two ranks computes its contiguous heads (per-head windows) through
+    the CUDA path; every row of every head is compared with the oracle.  The ranks
+    share the run's one GPU; their kernels are independent (no collective)."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from sparse_attention_video_tile_b200.build import build
+    build()
+    world = 2
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as mgr:
+        results = mgr.dict()
+        mp.start_processes(_gpu_rank_main, args=(world, _free_port(), results), nprocs=world, join=True,
+                           start_method="spawn")
+        res = dict(results)
+    covered = []
+    for r in range(world):
+        assert not isinstance(res[r], str), f"rank {r}: {res[r]}"
+        h0, h1, err, rel = res[r]
+        covered += list(range(h0, h1))
+        assert err <= 1e-2 and rel <= 5e-3, f"rank {r} heads [{h0}, {h1}): max abs {err:.3e}, rel {rel:.3e}"
+    assert covered == list(range(5))

@@ -10,6 +10,10 @@ This file is named to be collected last, so that a run stopping at the first
 failure has already run every other test.  It must pass on its own in a fresh
 process (the first call sets up the array's device address) and after the other
 tests.
+
+A kernel of this entry point that gives up on a bounded wait records it in the
+array's status word; sta_check_device_status reads and clears that word, and
+sta_selftest_bounded_wait runs a wait out through it.
 """
 import ctypes
 
@@ -59,6 +63,8 @@ def _check_against_allocating_entry(fn, cfg, seed):
     got = torch.full_like(qt, float("nan"))
     assert _call(fn, qt, kt, vt, got, cfg) == 0
     torch.cuda.synchronize()
+    # the call's status word (and the allocating path's) report no expired wait
+    assert sta.sta_check_device_status() == sta.STA_OK
     a = got.float().cpu().numpy().astype(np.float64)
     b = ref.float().cpu().numpy().astype(np.float64)
     assert np.all(np.isfinite(a))
@@ -85,3 +91,23 @@ def test_noalloc_rejects_schedule_larger_than_scratch(noalloc):
                  sta._windows(cfg.windows), ctypes.c_float(cfg.scale), torch.cuda.current_stream().cuda_stream)
     assert st == STA_ERR_SCRATCH
     assert sta.sta_status_str(st) == "STA_ERR_SCRATCH"
+
+
+def test_noalloc_timeouts_are_reported_and_cleared(noalloc):
+    # After a good call its status word is clear ...
+    _check_against_allocating_entry(noalloc, W.CONFIGS["tiny"], 11)
+    # ... a wait run out through every status word of the device (the no-alloc
+    # array's among them, now that it is set up) is reported ...
+    assert sta.sta_selftest_bounded_wait(20_000_000) == sta.STA_ERR_TIMEOUT
+    # ... and the check after it finds every word cleared.
+    assert sta.sta_check_device_status() == sta.STA_OK
+    # The next call still computes correctly and leaves its word clear.
+    _check_against_allocating_entry(noalloc, W.CONFIGS["small"], 12)
+
+
+def test_noalloc_after_shutdown_sets_up_again(noalloc):
+    _check_against_allocating_entry(noalloc, W.CONFIGS["small"], 13)
+    sta.sta_shutdown()
+    # the same configuration again: the set-up and the upload are redone
+    _check_against_allocating_entry(noalloc, W.CONFIGS["small"], 14)
+    _check_against_allocating_entry(noalloc, W.CONFIGS["small"], 15)
