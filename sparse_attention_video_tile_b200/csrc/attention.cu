@@ -35,7 +35,11 @@
 //     rescaled together, so O / l is unchanged); the other warp reads that
 //     before publishing its next block and redoes rows it computed against the
 //     old reference.  The epilogue adds the two warps' sums, divides and writes
-//     bf16 rows, each warp half of the head dimension.
+//     bf16 rows, each warp half of the head dimension;
+//   * warpgroup 2 (warps 8-11: the producer, the two issuers and one idle warp)
+//     lowers its register count with setmaxnreg and the two softmax warpgroups
+//     raise theirs to 224, so that a softmax thread holds half a row of S, the
+//     row's P and its state without spilling.
 //
 // Every barrier that is waited on with a parity can never run two phases ahead
 // of its waiter (the per-buffer S, P and P*V barriers, the Q pair, the ring).
@@ -62,7 +66,9 @@ namespace {
 
 using namespace ptx;
 
-constexpr int kThreads = 352;       // warps 0-7 softmax + epilogue, 8 producer, 9-10 MMA issuers
+constexpr int kThreads = 384;       // warps 0-7 softmax + epilogue, 8 producer, 9-10 MMA issuers, 11 idle
+constexpr int kRegsSoftmax = 224;   // setmaxnreg: warpgroups 0-1 (softmax) raise, warpgroup 2 lowers
+constexpr int kRegsOther = 56;
 constexpr int kProducerWarp = 8;
 constexpr int kPvWarp = 9;          // issues O += P V; also owns the TMEM allocation
 constexpr int kSWarp = 10;          // issues S = Q K^T
@@ -219,6 +225,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int kBoxes = D / 64;
   constexpr uint32_t kBlockBytes = S::kBlockBytes;
 
+  if (warp >= 8) setmaxnreg_dec<kRegsOther>();
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -371,7 +378,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait_drain(drain, 0, p.limit_ns);
     }
     __syncwarp();
-  } else {
+  } else if (warp < 8) {
+    setmaxnreg_inc<kRegsSoftmax>();
     // ------------------------------------------------------------ softmax + epilogue
     // Warps w and w+4 share the rows of TMEM lane quadrant w and take the blocks of
     // the CTA's stream alternately (block g by the warp with h = g mod 2), each
