@@ -33,6 +33,7 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "STA fwd ms & TFLOPS (attended) at 30×48×80, 24 heads, d=128; % of BF16 peak"
+DEFAULT_PATH = "three_call"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM bytes (read + write) per launch of the tiled-order attention kernel on the default
@@ -283,7 +284,30 @@ def run_ours(args, cfg):
             ev["a0"].append(a0)
             ev["a1"].append(a1)
 
-    step = step_fused if fused else step_three
+    kpad = torch.empty((cfg.batch, cfg.heads, sta.padded_rows(grid, tile), cfg.d), dtype=q.dtype, device=dev) \
+        if sta.raster_tile_ok(tile) else None
+    vpad = torch.empty_like(kpad) if kpad is not None else None
+
+    def step_mixed(record: bool, store=ev):
+        # k and v into the padded latent's tiled order (two launches), then the kernel
+        # that reads q and writes the output in raster order
+        if record:
+            e = {n: torch.cuda.Event(enable_timing=True) for n in ("r0", "r1", "a0", "a1")}
+            e["r0"].record(stream)
+        sta.sta_tile_reorder_padded(k, kpad, grid, tile, stream)
+        sta.sta_tile_reorder_padded(v, vpad, grid, tile, stream)
+        if record:
+            e["r1"].record(stream)
+            e["a0"].record(stream)
+        sta.sta_attention_fwd_mixed(q, kpad, vpad, out, grid, tile, wins, scale, stream)
+        if record:
+            e["a1"].record(stream)
+            for n in ("r0", "r1", "a0", "a1"):
+                store[n].append(e[n])
+
+    if args.path == "mixed" and kpad is None:
+        raise SystemExit("--path mixed needs a tile that splits into 128-row slabs of whole frames")
+    step = {"three_call": step_three, "fused": step_fused, "mixed": step_mixed}[args.path]
 
     def barrier():
         if world > 1:
@@ -319,10 +343,10 @@ def run_ours(args, cfg):
     # extra steps when the fused kernel was the step), and the other path's step time
     # (not part of `value`)
     hbm = load_peaks().get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"])
-    ev3 = ev if not fused else {n: [] for n in ("r0", "r1", "a0", "a1", "u0", "u1")}
+    ev3 = ev if args.path == "three_call" else {n: [] for n in ("r0", "r1", "a0", "a1", "u0", "u1")}
     three = None
     other = None
-    if fused and args.aux_steps > 0:
+    if args.path != "three_call" and args.aux_steps > 0:
         for _ in range(2):
             step_three(False)
         torch.cuda.synchronize()
@@ -338,6 +362,19 @@ def run_ours(args, cfg):
                  "tiled_attention_ms": att3_ms, "tiled_attention_tflops": flops / (att3_ms * 1e-3) / 1e12,
                  "reorder_ms_per_tensor": reo_ms, "reorder_gbs": reo_gbs, "reorder_frac_hbm": reo_gbs / hbm,
                  "unorder_ms": uno_ms, "unorder_gbs": 2 * tensor_bytes / (uno_ms * 1e-3) / 1e9}
+    mixed = None
+    if args.path != "mixed" and args.aux_steps > 0 and kpad is not None:
+        evm = {n: [] for n in ("r0", "r1", "a0", "a1")}
+        for _ in range(2):
+            step_mixed(False)
+        torch.cuda.synchronize()
+        for _ in range(args.aux_steps):
+            step_mixed(True, evm)
+        torch.cuda.synchronize()
+        m_re = statistics.median(a.elapsed_time(b) for a, b in zip(evm["r0"], evm["r1"]))
+        m_at = statistics.median(a.elapsed_time(b) for a, b in zip(evm["a0"], evm["a1"]))
+        mixed = {"steps": args.aux_steps, "step_ms": m_re + m_at, "padded_reorder_ms_k_and_v": m_re,
+                 "mixed_attention_ms": m_at, "mixed_attention_tflops": flops / (m_at * 1e-3) / 1e12}
     if not fused and args.aux_steps > 0 and sta.raster_tile_ok(tile):
         evf = {"a0": [], "a1": []}
         for _ in range(2):
@@ -456,23 +493,25 @@ def run_ours(args, cfg):
         # The attention kernel runs for ~10-20 ms at a time inside a timed loop of well
         # under a second, at the full SM clock: the burst bf16 figure is its peak.  The
         # sustained (seconds-long, power-capped) figure is kept beside it.
-        "roofline": {"bound": "tensor", "kernel": "sta_fwd_kernel" + ("<raster>" if fused else "<tiled>"),
+        "roofline": {"bound": "tensor", "kernel": "sta_fwd_kernel" + {"fused": "<raster>", "three_call": "<tiled>",
+                                                                      "mixed": "<mixed>"}[args.path],
                      "achieved": att_tflops, "peak": peak_b,
                      "unit": "TFLOP/s", "frac": att_tflops / peak_b, "traffic": traffic,
                      "peak_kind": f"bf16_tflops, burst ({peaks['_source']})",
                      "frac_of_sustained_peak": att_tflops / peak_s, "frac_of_2250_datasheet": att_tflops / 2250.0},
         "kernels": {"attention_ms": att_ms, "attention_ms_min": att_min, "attention_steps": len(att_list),
                     "attention_tflops": att_tflops,
-                    "path": "fused raster-order kernel, 1 launch per step" if fused else
-                            "reorder x3 + tiled attention + unorder, 5 launches per step",
-                    "three_call_path": three, "fused_path": other, "backward": backward,
+                    "path": {"fused": "fused raster-order kernel, 1 launch per step",
+                             "three_call": "reorder x3 + tiled attention + unorder, 5 launches per step",
+                             "mixed": "padded reorder of k and v + raster-q attention, 3 launches per step"}[args.path],
+                    "three_call_path": three, "fused_path": other, "mixed_path": mixed, "backward": backward,
                     "token_major_reorder": token_major},
         "cpu_baseline": cpu,
         "e2e": {"value": job_tflops(world, flops, e2e_ms), "unit": "TFLOPS", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": 3 * tensor_bytes, "d2h_bytes_per_step": tensor_bytes,
                 "steps": e2e_steps},
         "clocks": clk.summary(),
-        "gpu_launches": (1 if fused else 5) * args.steps,
+        "gpu_launches": {"fused": 1, "three_call": 5, "mixed": 3}[args.path] * args.steps,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -493,7 +532,10 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=512)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--fused", action="store_true",
-                    help="time the one-launch fused raster-order kernel as the step")
+                    help="time the one-launch fused raster-order kernel as the step (same as --path fused)")
+    ap.add_argument("--path", choices=["three_call", "fused", "mixed"], default=None,
+                    help="the forward timed as the step: reorder x3 + tiled attention + unorder (three_call), "
+                         "the one-launch raster kernel (fused), or padded reorder of k and v + the raster-q kernel (mixed)")
     ap.add_argument("--aux-steps", type=int, default=10,
                     help="extra steps of the path not timed as the step (0: none)")
     ap.add_argument("--backward-steps", type=int, default=5,
@@ -503,6 +545,9 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("at least 3 warm-up steps are required")
+    if args.path is None:
+        args.path = "fused" if args.fused else DEFAULT_PATH
+    args.fused = args.path == "fused"
     import workloads as W
     cfg = W.CONFIGS[args.config]
     if args.heads:

@@ -59,7 +59,8 @@ typedef enum {
   STA_ERR_CUDA = 8,      /* a CUDA runtime/driver call failed (message via sta_last_cuda_error) */
   STA_ERR_TIMEOUT = 9,   /* a kernel's bounded wait expired; the kernel gave up */
   STA_ERR_ARG = 10,      /* another argument is out of range (batch, heads, scale not finite ...) */
-  STA_ERR_SCRATCH = 11   /* the work schedule does not fit the fixed scratch of sta_attention_fwd_noalloc */
+  STA_ERR_SCRATCH = 11,  /* the work schedule does not fit the fixed scratch of sta_attention_fwd_noalloc */
+  STA_ERR_BOUNDS = 12    /* a device-side bounds check failed (libsta_checked.so only); the kernel skipped the access */
 } sta_status;
 
 /* Human-readable name of a status code.  Static storage; never NULL. */
@@ -219,6 +220,44 @@ sta_status sta_attention_fwd_raster(const void* q, const void* k, const void* v,
                                     void* stream);
 
 /*
+ * Tile reorder into the padded latent (raster -> tiled), for grids that need not
+ * be tile multiples ("padding with masking", review reply on input resolution).
+ * The latent is treated as padded up to the next tile multiple in every dimension:
+ * Lpad = ceil(T/tt)*tt * ceil(H/th)*th * ceil(W/tw)*tw rows per (batch, head).
+ *   src: device bf16 [batch_heads, T*H*W, d], raster order; 16-byte aligned.
+ *   dst: device bf16 [batch_heads, Lpad, d], tiled order of the padded latent;
+ *        the rows of pad tokens are written as zeros.  Must not overlap src.
+ * On tile-multiple grids the result equals sta_tile_reorder's.  Asynchronous on
+ * `stream`.
+ * Errors: NULL, ALIGN, ALIAS, SHAPE (nonpositive sizes, too large), HEADDIM, ARG,
+ * ARCH, CUDA.
+ */
+sta_status sta_tile_reorder_padded(const void* src, void* dst, int64_t batch_heads, int32_t d, sta_dim3 grid,
+                                   sta_dim3 tile, void* stream);
+
+/*
+ * STA forward with raster-order queries and output and tiled-order keys and
+ * values: the query blocks are read from raster order by the kernel's loads (one
+ * load per block of 128 queries, the same 5-D boxes as sta_attention_fwd_raster)
+ * and the output rows are written to raster order, while the key and value blocks,
+ * read once for every query block whose window holds them, come from tiled copies
+ * (sta_tile_reorder_padded), 128 contiguous rows each.  The grid need not be a
+ * tile multiple (padding with masking, as sta_attention_fwd_raster).
+ *   q, out: device bf16 [batch, heads, T*H*W, d], raster order, 16-byte aligned;
+ *   k_tiled, v_tiled: device bf16 [batch, heads, Lpad, d], tiled order of the
+ *   padded latent with zero pad rows, as written by sta_tile_reorder_padded;
+ *   out must not overlap q, k_tiled or v_tiled.
+ *   The tile must split into 128-row slabs of whole frames, as for
+ *   sta_attention_fwd_raster.
+ * Results equal sta_attention_fwd_raster's bit for bit (same schedule and
+ * arithmetic).  Same schedule caching and status reporting as sta_attention_fwd.
+ * Errors: NULL, ALIGN, ALIAS, SHAPE, WINDOW, HEADDIM, ARG, ARCH, CUDA.
+ */
+sta_status sta_attention_fwd_mixed(const void* q, const void* k_tiled, const void* v_tiled, void* out,
+                                   int32_t batch, int32_t heads, int32_t d, sta_dim3 grid, sta_dim3 tile,
+                                   const sta_dim3* window_per_head, float scale, void* stream);
+
+/*
  * sta_attention_fwd without any device allocation by the library.  The paper has
  * no counterpart: this entry point exists for callers that cannot let a library
  * call cudaMalloc - code running inside a memory pool or arena it must not
@@ -247,7 +286,9 @@ sta_status sta_attention_fwd_noalloc(const void* q, const void* k, const void* v
 /*
  * Synchronises `stream` and reports whether any kernel of this library on the
  * current device gave up on a bounded wait since the last check
- * (STA_ERR_TIMEOUT), then clears the flag.  The flags read are the allocating
+ * (STA_ERR_TIMEOUT) or, in the checked build (libsta_checked.so, compiled with
+ * STA_DEVICE_CHECKS=1), failed a bounds check on an index taken from its work
+ * schedule (STA_ERR_BOUNDS, which takes precedence), then clears the flag.  The flags read are the allocating
  * entry points' status word and, once sta_attention_fwd_noalloc has run on the
  * device, that entry point's own.  Returns STA_ERR_CUDA if the stream has a
  * pending CUDA error.

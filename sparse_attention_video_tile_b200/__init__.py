@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(_HERE, "libsta.so")
 STATUS_NAMES = {
     0: "STA_OK", 1: "STA_ERR_NULL", 2: "STA_ERR_ALIGN", 3: "STA_ERR_ALIAS", 4: "STA_ERR_SHAPE",
     5: "STA_ERR_WINDOW", 6: "STA_ERR_HEADDIM", 7: "STA_ERR_ARCH", 8: "STA_ERR_CUDA",
-    9: "STA_ERR_TIMEOUT", 10: "STA_ERR_ARG", 11: "STA_ERR_SCRATCH",
+    9: "STA_ERR_TIMEOUT", 10: "STA_ERR_ARG", 11: "STA_ERR_SCRATCH", 12: "STA_ERR_BOUNDS",
 }
 STA_OK, STA_ERR_TIMEOUT = 0, 9
 
@@ -63,6 +63,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "sta_tile_unorder_tokens": (ctypes.c_int, [P, P, I32, I32, I32, D3, D3, P]),
         "sta_attention_fwd": (ctypes.c_int, [P, P, P, P, I32, I32, I32, D3, D3, ctypes.POINTER(D3), F, P]),
         "sta_attention_fwd_raster": (ctypes.c_int, [P, P, P, P, I32, I32, I32, D3, D3, ctypes.POINTER(D3), F, P]),
+        "sta_attention_fwd_mixed": (ctypes.c_int, [P, P, P, P, I32, I32, I32, D3, D3, ctypes.POINTER(D3), F, P]),
+        "sta_tile_reorder_padded": (ctypes.c_int, [P, P, I64, I32, D3, D3, P]),
         "sta_attention_fwd_lse": (ctypes.c_int, [P, P, P, P, P, I32, I32, I32, D3, D3, ctypes.POINTER(D3), F, P]),
         "sta_attention_bwd": (ctypes.c_int, [P, P, P, P, P, P, P, P, P, I32, I32, I32, D3, D3, ctypes.POINTER(D3), F, P]),
         "sta_check_device_status": (ctypes.c_int, [P]),
@@ -302,6 +304,45 @@ def sta_attention_fwd_raster(q, k, v, out, grid, tile, window_per_head, scale: f
     _check(st, "sta_attention_fwd_raster")
 
 
+def padded_rows(grid, tile) -> int:
+    """Rows per (batch, head) of the latent padded up to tile multiples."""
+    return int(np.prod([-(-int(a) // int(b)) * int(b) for a, b in zip(grid, tile)]))
+
+
+def sta_tile_reorder_padded(src, dst, grid, tile, stream=None) -> None:
+    """Raster [.., T*H*W, d] -> tiled order of the padded latent [.., Lpad, d], pad rows zero."""
+    d = int(src.shape[-1])
+    lead = tuple(int(x) for x in src.shape[:-2])
+    if tuple(dst.shape) != lead + (padded_rows(grid, tile), d):
+        raise ValueError(f"dst must be {lead + (padded_rows(grid, tile), d)}")
+    bh = int(np.prod(lead)) if lead else 1
+    st = load_library().sta_tile_reorder_padded(_tensor_ptr(src, "src"), _tensor_ptr(dst, "dst"), bh, d,
+                                                _d3(grid), _d3(tile), _stream(stream))
+    _check(st, "sta_tile_reorder_padded")
+
+
+def sta_attention_fwd_mixed(q, k_tiled, v_tiled, out, grid, tile, window_per_head, scale: float, stream=None) -> None:
+    """STA forward with raster-order q and out [B, heads, T*H*W, d] and k, v in the tiled
+    order of the padded latent [B, heads, Lpad, d] (``sta_tile_reorder_padded``)."""
+    if q.dim() != 4:
+        raise ValueError("q must be [batch, heads, L, d]")
+    B, Hn, L, d = (int(x) for x in q.shape)
+    if tuple(out.shape) != tuple(q.shape):
+        raise ValueError("out must be shaped like q")
+    for name, t in (("k_tiled", k_tiled), ("v_tiled", v_tiled)):
+        if tuple(t.shape) != (B, Hn, padded_rows(grid, tile), d):
+            raise ValueError(f"{name} must be [B, heads, Lpad, d]")
+    if len(window_per_head) != Hn:
+        raise ValueError("one window per head is required")
+    if L != int(np.prod([int(x) for x in grid])):
+        raise ValueError("L must equal T*H*W")
+    st = load_library().sta_attention_fwd_mixed(_tensor_ptr(q, "q"), _tensor_ptr(k_tiled, "k_tiled"),
+                                                _tensor_ptr(v_tiled, "v_tiled"), _tensor_ptr(out, "out"), B, Hn, d,
+                                                _d3(grid), _d3(tile), _windows(window_per_head), float(scale),
+                                                _stream(stream))
+    _check(st, "sta_attention_fwd_mixed")
+
+
 def raster_tile_ok(tile) -> bool:
     """Whether sta_attention_fwd_raster accepts this tile (128-row slabs of whole frames)."""
     tt, th, tw = (int(x) for x in tile)
@@ -329,10 +370,17 @@ def sta_shutdown() -> None:
 
 
 def sta_forward(q, k, v, grid, tile, window_per_head, scale: Optional[float] = None,
-                stream=None, workspace: Optional[Tuple] = None, fused: Optional[bool] = None):
+                stream=None, workspace: Optional[Tuple] = None, fused: Optional[bool] = None,
+                path: Optional[str] = None):
     """Full STA forward on raster-order [B, heads, L, d] bf16 CUDA tensors.
 
-    Two ways, same result:
+    Three ways (``path``), same result:
+
+    * "mixed": k and v are reordered into the padded latent's tiled order (two
+      launches of ``sta_tile_reorder_padded``), then ``sta_attention_fwd_mixed``
+      reads q and writes out in raster order.  Needs ``raster_tile_ok`` and two
+      scratch tensors [B, heads, Lpad, d] (``workspace`` may hold them); handles
+      grids that are not tile multiples.
 
     * fused: one call does everything (``sta_attention_fwd_raster``: tile reorder in
       the kernel's loads and stores).  Needs a tile that splits into 128-row slabs
@@ -344,20 +392,36 @@ def sta_forward(q, k, v, grid, tile, window_per_head, scale: Optional[float] = N
       apply (the tiled kernel's K/V loads are plain 3-D boxes of 128 contiguous
       rows, the fused kernel's are 5-D boxes of whole frames).
 
-    ``fused=None`` takes the fused call only when the grid is not a tile multiple.
+    ``path`` is "mixed", "fused" (the one-launch raster call) or "three_call";
+    ``fused=True`` / ``fused=False`` select "fused" / "three_call".  By default the
+    fused call is taken only when the grid is not a tile multiple.
     Returns the raster-order output, allocated on ``stream``: use it on another
     stream only after synchronising with that one.
     """
     import torch
     if scale is None:
         scale = 1.0 / float(q.shape[-1]) ** 0.5
-    if fused is None:
-        multiple = all(int(a) % int(b) == 0 for a, b in zip(grid, tile))
-        fused = not multiple and raster_tile_ok(tile)
+    if path is None:
+        if fused is None:
+            multiple = all(int(a) % int(b) == 0 for a, b in zip(grid, tile))
+            fused = not multiple and raster_tile_ok(tile)
+        path = "fused" if fused else "three_call"
+    if path not in ("mixed", "fused", "three_call"):
+        raise ValueError(f"unknown path {path!r}")
     with _stream_context(stream):
         out = torch.empty_like(q)
-        if fused:
+        if path == "fused":
             sta_attention_fwd_raster(q, k, v, out, grid, tile, window_per_head, scale, stream)
+            return out
+        if path == "mixed":
+            B, Hn, _, d = (int(x) for x in q.shape)
+            if workspace is None:
+                workspace = tuple(torch.empty((B, Hn, padded_rows(grid, tile), d), dtype=q.dtype, device=q.device)
+                                  for _ in range(2))
+            kt, vt = workspace[:2]
+            sta_tile_reorder_padded(k, kt, grid, tile, stream)
+            sta_tile_reorder_padded(v, vt, grid, tile, stream)
+            sta_attention_fwd_mixed(q, kt, vt, out, grid, tile, window_per_head, scale, stream)
             return out
         if workspace is None:
             workspace = tuple(torch.empty_like(q) for _ in range(4))

@@ -1,4 +1,6 @@
-"""Builds the in-tree CUDA library ``libsta.so`` for sm_100a with nvcc.
+"""Builds the in-tree CUDA library ``libsta.so`` for sm_100a with nvcc, and its
+checked twin ``libsta_checked.so`` (device-side bounds checks on the forward
+kernel's schedule-derived indices, for tests).
 
 Usage: ``python -m sparse_attention_video_tile_b200.build [--verbose]``.
 The library lands next to this file so the Python binding finds it; it is
@@ -33,38 +35,53 @@ def nvcc() -> str:
     return path
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+LIB_CHECKED = os.path.join(HERE, "libsta_checked.so")
+
+
+def _stale(lib: str) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = [os.path.join(CSRC, s) for s in SOURCES + HEADERS] + [os.path.join(INCLUDE, "sta.h")]
     return any(os.path.getmtime(p) > t for p in deps)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile every source and link libsta.so; returns the library path."""
-    if not force and not _stale():
-        return LIB
-    os.makedirs(BUILD_DIR, exist_ok=True)
-    objs = []
+def _build_lib(lib: str, obj_dir: str, defines, verbose: bool) -> None:
+    os.makedirs(obj_dir, exist_ok=True)
+    objs, procs = [], []
     for src in SOURCES:
-        obj = os.path.join(BUILD_DIR, src + ".o")
-        cmd = [nvcc(), *ARCH, *NVCC_FLAGS, "-I", INCLUDE, "-c", os.path.join(CSRC, src), "-o", obj]
+        obj = os.path.join(obj_dir, src + ".o")
+        cmd = [nvcc(), *ARCH, *NVCC_FLAGS, *defines, "-I", INCLUDE, "-c", os.path.join(CSRC, src), "-o", obj]
         if verbose and src.endswith(".cu"):
             cmd += ["-Xptxas", "-v"]
-        r = subprocess.run(cmd, capture_output=True, text=True)
-        if verbose or r.returncode != 0:
-            sys.stderr.write(r.stdout + r.stderr)
-        if r.returncode != 0:
-            raise RuntimeError(f"nvcc failed on {src}")
+        procs.append((src, subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.STDOUT, text=True)))
         objs.append(obj)
-    tmp = LIB + ".tmp"
+    failed = []
+    for src, pr in procs:
+        out = pr.communicate()[0]
+        if verbose or pr.returncode != 0:
+            sys.stderr.write(out)
+        if pr.returncode != 0:
+            failed.append(src)
+    if failed:
+        raise RuntimeError(f"nvcc failed on {', '.join(failed)}")
+    tmp = lib + ".tmp"
     cmd = [nvcc(), *ARCH, "-shared", "-o", tmp, *objs, "-lcudart"]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         sys.stderr.write(r.stdout + r.stderr)
-        raise RuntimeError("linking libsta.so failed")
-    os.replace(tmp, LIB)
+        raise RuntimeError(f"linking {os.path.basename(lib)} failed")
+    os.replace(tmp, lib)
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    """Compile every source and link libsta.so and its checked twin
+    libsta_checked.so (device-side bounds checks, STA_DEVICE_CHECKS=1); returns
+    the path of libsta.so."""
+    if force or _stale(LIB):
+        _build_lib(LIB, BUILD_DIR, [], verbose)
+    if force or _stale(LIB_CHECKED):
+        _build_lib(LIB_CHECKED, os.path.join(BUILD_DIR, "checked"), ["-DSTA_DEVICE_CHECKS=1"], verbose)
     return LIB
 
 

@@ -3,6 +3,7 @@
 #include <cuda_runtime.h>
 
 #include <cmath>
+#include <cstdlib>
 #include <cstring>
 #include <list>
 #include <map>
@@ -128,6 +129,13 @@ sta_status get_schedule(DeviceState* st, const Geometry& g, int32_t batch, int32
     build_schedule(g, batch, heads, windows, &cs->host);
   for (const WorkItem& w : cs->host.items)
     if (w.kv_len < 1) return STA_ERR_ARG;  // cannot happen: a tile always sees itself
+#if STA_DEVICE_CHECKS
+  // Checked builds only: STA_CHECKS_PLANT_BAD_ROW=1 plants a key-block row far past
+  // the tensor in the schedule, so that a test can see the device check catch it.
+  // (A tensor-map load at such a row would read zeros, not fault.)
+  if (const char* plant = std::getenv("STA_CHECKS_PLANT_BAD_ROW"))
+    if (plant[0] == '1' && !cs->host.kv_rows.empty()) cs->host.kv_rows[0] = static_cast<int32_t>(g.Lpad) + 64 * kBlockRows;
+#endif
   cudaError_t e;
   if ((e = upload(&cs->d_items, cs->host.items)) != cudaSuccess ||
       (e = upload(&cs->d_kv_rows, cs->host.kv_rows)) != cudaSuccess ||
@@ -186,6 +194,7 @@ const char* sta_status_str(sta_status s) {
     case STA_ERR_TIMEOUT: return "STA_ERR_TIMEOUT";
     case STA_ERR_ARG: return "STA_ERR_ARG";
     case STA_ERR_SCRATCH: return "STA_ERR_SCRATCH";
+    case STA_ERR_BOUNDS: return "STA_ERR_BOUNDS";
   }
   return "STA_ERR_UNKNOWN";
 }
@@ -331,6 +340,7 @@ sta_status attention_fwd_impl(const void* q, const void* k, const void* v, void*
   if ((s = get_schedule(st, g, batch, heads, window_per_head, 0, &cs)) != STA_OK) return s;
   DeviceSchedule ds{cs->d_items, cs->d_kv_rows, cs->d_head_win, static_cast<int32_t>(cs->host.items.size()),
                     cs->host.masked};
+  ds.n_kv_rows = static_cast<int32_t>(cs->host.kv_rows.size());
   cudaError_t e = launch_attention(q, k, v, out, batch, heads, d, g, ds, scale, st->d_err, kWaitLimitNs,
                                    static_cast<cudaStream_t>(stream), lse);
   return e == cudaSuccess ? STA_OK : cuda_fail(e);
@@ -436,20 +446,20 @@ sta_status sta_attention_fwd_raster(const void* q, const void* k, const void* v,
   CachedSchedule* cs = nullptr;
   if ((s = get_schedule(st, g, batch, heads, window_per_head, 1, &cs)) != STA_OK) return s;
   DeviceSchedule ds{cs->d_items, cs->d_kv_rows, cs->d_head_win, static_cast<int32_t>(cs->host.items.size()), false,
-                    cs->d_kv_mask_id, cs->d_kv_masks};
+                    cs->d_kv_mask_id, cs->d_kv_masks, static_cast<int32_t>(cs->host.kv_rows.size()),
+                    static_cast<int32_t>(cs->host.kv_masks.size() / 4)};
   cudaError_t e = launch_attention_raster(q, k, v, out, batch, heads, d, g, ds, scale, st->d_err, kWaitLimitNs,
                                           static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? STA_OK : cuda_fail(e);
 }
 
 namespace {
-// Reads a device status word; if it is set, clears it.  *set tells which.
-sta_status read_and_clear(int32_t* word, bool* set) {
-  int32_t flag = 0;
-  cudaError_t e = cudaMemcpy(&flag, word, sizeof(flag), cudaMemcpyDeviceToHost);
+// Reads a device status word into *flag; if it is set, clears it.  A flag is
+// 0x100 | site for an expired wait and 0x200 | code for a failed device check.
+sta_status read_and_clear(int32_t* word, int32_t* flag) {
+  cudaError_t e = cudaMemcpy(flag, word, sizeof(int32_t), cudaMemcpyDeviceToHost);
   if (e != cudaSuccess) return cuda_fail(e);
-  *set = flag != 0;
-  if (*set && (e = cudaMemset(word, 0, sizeof(int32_t))) != cudaSuccess) return cuda_fail(e);
+  if (*flag != 0 && (e = cudaMemset(word, 0, sizeof(int32_t))) != cudaSuccess) return cuda_fail(e);
   return STA_OK;
 }
 
@@ -467,6 +477,63 @@ int status_words(int dev, int32_t* words[2]) {
 }
 }  // namespace
 
+sta_status sta_tile_reorder_padded(const void* src, void* dst, int64_t batch_heads, int32_t d, sta_dim3 grid,
+                                   sta_dim3 tile, void* stream) {
+  if (!src || !dst) return STA_ERR_NULL;
+  if (!aligned16(src) || !aligned16(dst)) return STA_ERR_ALIGN;
+  if (d != 64 && d != 128) return STA_ERR_HEADDIM;
+  Geometry g;
+  sta_status s = make_geometry_padded(grid, tile, &g);
+  if (s != STA_OK) return s;
+  if (batch_heads < 0 || batch_heads > (int64_t(1) << 31)) return STA_ERR_ARG;
+  const char* a = static_cast<const char*>(src);
+  const char* b = static_cast<const char*>(dst);
+  if (batch_heads > 0 && a < b + batch_heads * g.Lpad * d * 2 && b < a + batch_heads * g.L * d * 2) return STA_ERR_ALIAS;
+  if ((s = check_device(nullptr)) != STA_OK) return s;
+  cudaError_t e = launch_reorder_padded(src, dst, batch_heads, d, g, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? STA_OK : cuda_fail(e);
+}
+
+sta_status sta_attention_fwd_mixed(const void* q, const void* k_tiled, const void* v_tiled, void* out, int32_t batch,
+                                   int32_t heads, int32_t d, sta_dim3 grid, sta_dim3 tile,
+                                   const sta_dim3* window_per_head, float scale, void* stream) {
+  if (!q || !k_tiled || !v_tiled || !out || !window_per_head) return STA_ERR_NULL;
+  if (!aligned16(q) || !aligned16(k_tiled) || !aligned16(v_tiled) || !aligned16(out)) return STA_ERR_ALIGN;
+  if (d != 64 && d != 128) return STA_ERR_HEADDIM;
+  Geometry g;
+  sta_status s = make_geometry_padded(grid, tile, &g);
+  if (s != STA_OK) return s;
+  if (!raster_tile_ok(g.tt, g.th, g.tw) || g.ntile % kBlockRows != 0) return STA_ERR_SHAPE;
+  if (batch < 1 || heads < 1 || static_cast<int64_t>(batch) * heads > (int64_t(1) << 24)) return STA_ERR_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return STA_ERR_ARG;
+  for (int32_t h = 0; h < heads; ++h)
+    if (window_per_head[h].t < 1 || window_per_head[h].h < 1 || window_per_head[h].w < 1) return STA_ERR_WINDOW;
+  const int64_t rows = static_cast<int64_t>(batch) * heads;
+  const int64_t raster_bytes = rows * g.L * d * 2, tiled_bytes = rows * g.Lpad * d * 2;
+  auto hit = [](const void* x, int64_t nx, const void* y, int64_t ny) {
+    const char* a = static_cast<const char*>(x);
+    const char* b = static_cast<const char*>(y);
+    return a < b + ny && b < a + nx;
+  };
+  if (hit(out, raster_bytes, q, raster_bytes) || hit(out, raster_bytes, k_tiled, tiled_bytes) ||
+      hit(out, raster_bytes, v_tiled, tiled_bytes))
+    return STA_ERR_ALIAS;
+  int dev = 0;
+  if ((s = check_device(&dev)) != STA_OK) return s;
+
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState* st = nullptr;
+  if ((s = device_state(dev, &st)) != STA_OK) return s;
+  CachedSchedule* cs = nullptr;
+  if ((s = get_schedule(st, g, batch, heads, window_per_head, 1, &cs)) != STA_OK) return s;
+  DeviceSchedule ds{cs->d_items, cs->d_kv_rows, cs->d_head_win, static_cast<int32_t>(cs->host.items.size()), false,
+                    cs->d_kv_mask_id, cs->d_kv_masks, static_cast<int32_t>(cs->host.kv_rows.size()),
+                    static_cast<int32_t>(cs->host.kv_masks.size() / 4)};
+  cudaError_t e = launch_attention_mixed(q, k_tiled, v_tiled, out, batch, heads, d, g, ds, scale, st->d_err,
+                                         kWaitLimitNs, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? STA_OK : cuda_fail(e);
+}
+
 sta_status sta_check_device_status(void* stream) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -474,14 +541,15 @@ sta_status sta_check_device_status(void* stream) {
   if ((e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream))) != cudaSuccess) return cuda_fail(e);
   int32_t* words[2];
   const int n = status_words(dev, words);
-  bool any = false;
+  sta_status result = STA_OK;
   for (int i = 0; i < n; ++i) {
-    bool set = false;
-    sta_status s = read_and_clear(words[i], &set);
+    int32_t flag = 0;
+    sta_status s = read_and_clear(words[i], &flag);
     if (s != STA_OK) return s;
-    any = any || set;
+    if ((flag & 0x200) != 0) result = STA_ERR_BOUNDS;
+    else if (flag != 0 && result == STA_OK) result = STA_ERR_TIMEOUT;
   }
-  return any ? STA_ERR_TIMEOUT : STA_OK;
+  return result;
 }
 
 sta_status sta_selftest_bounded_wait(uint64_t limit_ns, void* stream) {
@@ -505,9 +573,9 @@ sta_status sta_selftest_bounded_wait(uint64_t limit_ns, void* stream) {
   if ((e = cudaStreamSynchronize(cs)) != cudaSuccess) return cuda_fail(e);
   bool all = n > 0;
   for (int i = 0; i < n; ++i) {
-    bool set = false;
-    if ((s = read_and_clear(words[i], &set)) != STA_OK) return s;
-    all = all && set;
+    int32_t flag = 0;
+    if ((s = read_and_clear(words[i], &flag)) != STA_OK) return s;
+    all = all && (flag & 0x100) != 0;
   }
   return all ? STA_ERR_TIMEOUT : STA_OK;
 }

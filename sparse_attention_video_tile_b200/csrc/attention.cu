@@ -61,10 +61,21 @@
 #include "internal.h"
 #include "ptx.cuh"
 
+// Builds with STA_DEVICE_CHECKS=1 (the checked library) test every index the
+// kernel takes from the schedule or computes from it (work items, key-block rows,
+// mask ids, output rows) before using it.  A failed check records 0x200 | code in
+// the status word, sets the CTA's abort flag and skips the access; the pipeline
+// then drains as after an expired wait.
+#ifndef STA_DEVICE_CHECKS
+#define STA_DEVICE_CHECKS 0
+#endif
+
 namespace sta {
 namespace {
 
 using namespace ptx;
+
+constexpr bool kChecks = STA_DEVICE_CHECKS != 0;
 
 constexpr int kThreads = 384;       // warps 0-7 softmax + epilogue, 8 producer, 9-10 MMA issuers, 11 idle
 constexpr int kRegsSoftmax = 224;   // setmaxnreg: warpgroups 0-1 (softmax) raise, warpgroup 2 lowers
@@ -96,6 +107,11 @@ struct FwdParams {
   int32_t* err;
   uint64_t limit_ns;
   float* lse;                // per-row log-sum-exp (natural log), same row indexing as out, or null
+  // sizes for the device checks
+  int32_t n_kv_rows;         // entries of kv_rows (and kv_mask_id)
+  int32_t n_masks;           // 128-bit masks in kv_masks
+  int32_t n_bh;              // batch * heads
+  int32_t rows;              // rows per (batch, head) of the tiled order the schedule indexes
 };
 
 template <int D>
@@ -171,7 +187,12 @@ struct BlockCursor {
   }
 };
 
-template <int D, bool MASKED, int POLY8, bool RASTER>
+// Layout of the tensors the kernel reads and writes (LAYOUT template argument).
+constexpr int kTiled = 0;    // q, k, v, out in tiled order
+constexpr int kRaster = 1;   // q, k, v, out in raster order: 5-D boxes, raster output rows
+constexpr int kMixed = 2;    // q and out in raster order, k and v in the padded latent's tiled order
+
+template <int D, bool MASKED, int POLY8, int LAYOUT>
 __global__ void __launch_bounds__(kThreads, 1)
     sta_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -234,9 +255,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tm_v);
       uint32_t kv_seq = 0, q_loads[2] = {0, 0};
       bool ok = true;
-      // one 128-row block (Q into buffer `dst`, or K/V into the next ring stage)
-      auto tma_block = [&](uint32_t dst, const CUtensorMap* m, uint32_t full, int32_t row, int32_t bh) {
-        if constexpr (RASTER) {
+      // one 128-row block (Q into buffer `dst`, or K/V into the next ring stage);
+      // `raster`: the tensor is in raster order, read as 5-D boxes
+      auto tma_block = [&](uint32_t dst, const CUtensorMap* m, uint32_t full, int32_t row, int32_t bh, bool raster) {
+        if (raster) {
           const SlabCoord c = slab_coord(p, row);
           for (int b = 0; b < kBoxes; ++b) tma_load_5d(dst + b * kBoxBytes, m, full, b * 64, c.w, c.h, c.t, bh);
         } else {
@@ -248,20 +270,45 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(sb + S::kKvEmpty + 8 * st, ((kv_seq / kStages) & 1) ^ 1, wc, 2)) return false;
         const uint32_t full = sb + S::kKvFull + 8 * st;
         mbar_arrive_expect_tx(full, kBlockBytes);
-        tma_block(sb + S::kStage0 + st * kBlockBytes, m, full, row, bh);
+        tma_block(sb + S::kStage0 + st * kBlockBytes, m, full, row, bh, LAYOUT == kRaster);
         ++kv_seq;
         return true;
       };
+      // failed device check: record it and stop; the CTA drains as after an expired wait
+      auto fail = [&](int code) {
+        atomicCAS(p.err, 0, 0x200 | code);
+        *abort_flag = 1;
+      };
+      // row of key block j of the cursor's item, or -1 after a failed check
+      auto kv_row = [&](const BlockCursor& c, int code) -> int32_t {
+        const int32_t idx = c.it.kv_off + c.j;
+        if (kChecks && !(idx >= 0 && idx < p.n_kv_rows)) {
+          fail(code);
+          return -1;
+        }
+        const int32_t row = p.kv_rows[idx];
+        if (kChecks && !(row >= 0 && row < p.rows && row % kBlockRows == 0)) {
+          fail(code + 1);
+          return -1;
+        }
+        return row;
+      };
       // K of block (k, j), preceded by the item's Q when j = 0
       auto load_k = [&](const BlockCursor& c) -> bool {
+        if (kChecks && !(c.it.bh >= 0 && c.it.bh < p.n_bh && c.it.q_row0 >= 0 && c.it.q_row0 < p.rows &&
+                         c.it.q_row0 % kBlockRows == 0 && c.it.kv_len >= 1)) {
+          fail(1);
+          return false;
+        }
         if (c.j == 0) {
           const int qb = c.k % S::kQBufs;
           if (!mbar_wait(sb + S::kQEmpty + 8 * qb, ((c.k / S::kQBufs) & 1) ^ 1, wc, 1)) return false;
           mbar_arrive_expect_tx(sb + S::kQFull + 8 * qb, kBlockBytes);
-          tma_block(sb + S::kQ + qb * kBlockBytes, &tm_q, sb + S::kQFull + 8 * qb, c.it.q_row0, c.it.bh);
+          tma_block(sb + S::kQ + qb * kBlockBytes, &tm_q, sb + S::kQFull + 8 * qb, c.it.q_row0, c.it.bh, LAYOUT != kTiled);
           ++q_loads[qb];
         }
-        return load_ring(&tm_k, p.kv_rows[c.it.kv_off + c.j], c.it.bh);
+        const int32_t row = kv_row(c, 2);
+        return row >= 0 && load_ring(&tm_k, row, c.it.bh);
       };
       // Order of the loads: K_0, K_1, K_2, then V_g, K_g+3 for g = 0, 1, ... (the S
       // issuer needs K three blocks ahead of the P V issuer's V).
@@ -273,7 +320,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         kc.next(p);
       }
       while (ok && !vc.done) {
-        ok = load_ring(&tm_v, p.kv_rows[vc.it.kv_off + vc.j], vc.it.bh);
+        const int32_t row = kv_row(vc, 4);
+        ok = row >= 0 && load_ring(&tm_v, row, vc.it.bh);
         vc.next(p);
         if (ok && !kc.done) {
           ok = load_k(kc);
@@ -432,6 +480,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         m_run = -INFINITY;
         l_run = 0.f;
         have_m = false;
+        if (kChecks && !(item.bh >= 0 && item.bh < p.n_bh)) {
+          atomicCAS(p.err, 0, 0x200 | 7);
+          *abort_flag = 1;
+          break;
+        }
         if (MASKED) {
           const int head = item.bh % p.heads;
           const int32_t et = p.head_win[head * 4 + 0], eh = p.head_win[head * 4 + 1], ew = p.head_win[head * 4 + 2];
@@ -454,7 +507,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t m = 0xffffffffu;
           if (pad_masks) {
             // padded latent: keys of pad tokens in this block do not exist
-            const int32_t mid = p.kv_mask_id[item.kv_off + j];
+            int32_t mid = p.kv_mask_id[item.kv_off + j];
+            if (kChecks && mid >= p.n_masks) {
+              atomicCAS(p.err, 0, 0x200 | 6);
+              *abort_flag = 1;
+              mid = -1;
+            }
             if (mid >= 0) m = p.kv_masks[4 * mid + c];
           }
           if (MASKED) {
@@ -624,7 +682,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float inv_l = 1.0f / l_tot;
         const int32_t qrow = item.q_row0 + row;
         int64_t out_row = -1;  // destination row, or -1 for no real token
-        if constexpr (RASTER) {
+        if constexpr (LAYOUT != kTiled) {
           const int32_t tile = qrow / p.ntile, local = qrow - tile * p.ntile;
           const int32_t at = tile / (p.nH * p.nW), ah = (tile / p.nW) % p.nH, aw = tile % p.nW;
           const int32_t t = at * p.tt + local / (p.th * p.tw);
@@ -634,6 +692,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             out_row = ((static_cast<int64_t>(item.bh) * p.T + t) * p.H + hh) * p.W + w;
         } else if (qrow < p.L) {
           out_row = static_cast<int64_t>(item.bh) * p.L + qrow;
+        }
+        if (kChecks && out_row >= static_cast<int64_t>(p.n_bh) * (LAYOUT != kTiled ? p.T * p.H * p.W : p.L)) {
+          atomicCAS(p.err, 0, 0x200 | 8);
+          *abort_flag = 1;
+          out_row = -1;
         }
         // log of the row's sum of exp(scale * s): reference max plus log of the sum
         // taken against it, from log2 units to natural log
@@ -734,10 +797,10 @@ bool make_tmap_raster(CUtensorMap* m, const void* base, int64_t bh, const Geomet
   return r == CUDA_SUCCESS;
 }
 
-template <int D, bool MASKED, int POLY8, bool RASTER>
+template <int D, bool MASKED, int POLY8, int LAYOUT>
 cudaError_t launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
                      cudaStream_t stream) {
-  auto kern = sta_fwd_kernel<D, MASKED, POLY8, RASTER>;
+  auto kern = sta_fwd_kernel<D, MASKED, POLY8, LAYOUT>;
   const int smem = Smem<D>::kDynBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -769,16 +832,16 @@ int exp_poly8() {
   return v;
 }
 
-template <int D, bool MASKED, bool RASTER>
+template <int D, bool MASKED, int LAYOUT>
 cudaError_t launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
                      cudaStream_t stream) {
-  if (MASKED) return launch_t<D, MASKED, 0, RASTER>(tq, tk, tv, p, stream);
-  if (exp_poly8() == 1) return launch_t<D, MASKED, 1, RASTER>(tq, tk, tv, p, stream);
-  return launch_t<D, MASKED, 0, RASTER>(tq, tk, tv, p, stream);
+  if (MASKED) return launch_t<D, MASKED, 0, LAYOUT>(tq, tk, tv, p, stream);
+  if (exp_poly8() == 1) return launch_t<D, MASKED, 1, LAYOUT>(tq, tk, tv, p, stream);
+  return launch_t<D, MASKED, 0, LAYOUT>(tq, tk, tv, p, stream);
 }
 
-FwdParams make_params(void* out, int32_t heads, const Geometry& g, const DeviceSchedule& s, float scale,
-                      int32_t* err_flag, uint64_t limit_ns) {
+FwdParams make_params(void* out, int32_t batch_heads, int32_t heads, const Geometry& g, const DeviceSchedule& s,
+                      float scale, int32_t* err_flag, uint64_t limit_ns) {
   FwdParams p;
   p.items = s.items;
   p.kv_rows = s.kv_rows;
@@ -798,6 +861,10 @@ FwdParams make_params(void* out, int32_t heads, const Geometry& g, const DeviceS
   p.err = err_flag;
   p.limit_ns = limit_ns;
   p.lse = nullptr;
+  p.n_kv_rows = s.n_kv_rows;
+  p.n_masks = s.n_masks;
+  p.n_bh = batch_heads;
+  p.rows = static_cast<int32_t>(g.Lpad);
   return p;
 }
 
@@ -810,11 +877,11 @@ cudaError_t launch_attention(const void* q, const void* k, const void* v, void* 
   CUtensorMap tq, tk, tv;
   if (!make_tmap(&tq, q, bh, g.L, d) || !make_tmap(&tk, k, bh, g.L, d) || !make_tmap(&tv, v, bh, g.L, d))
     return cudaErrorInvalidValue;
-  FwdParams p = make_params(out, heads, g, s, scale, err_flag, limit_ns);
+  FwdParams p = make_params(out, static_cast<int32_t>(bh), heads, g, s, scale, err_flag, limit_ns);
   p.lse = lse;
   if (d == 128)
-    return s.masked ? launch_d<128, true, false>(tq, tk, tv, p, stream) : launch_d<128, false, false>(tq, tk, tv, p, stream);
-  return s.masked ? launch_d<64, true, false>(tq, tk, tv, p, stream) : launch_d<64, false, false>(tq, tk, tv, p, stream);
+    return s.masked ? launch_d<128, true, kTiled>(tq, tk, tv, p, stream) : launch_d<128, false, kTiled>(tq, tk, tv, p, stream);
+  return s.masked ? launch_d<64, true, kTiled>(tq, tk, tv, p, stream) : launch_d<64, false, kTiled>(tq, tk, tv, p, stream);
 }
 
 cudaError_t launch_attention_raster(const void* q, const void* k, const void* v, void* out, int32_t batch,
@@ -827,9 +894,24 @@ cudaError_t launch_attention_raster(const void* q, const void* k, const void* v,
   if (!make_tmap_raster(&tq, q, bh, g, d, bt) || !make_tmap_raster(&tk, k, bh, g, d, bt) ||
       !make_tmap_raster(&tv, v, bh, g, d, bt))
     return cudaErrorInvalidValue;
-  const FwdParams p = make_params(out, heads, g, s, scale, err_flag, limit_ns);
-  if (d == 128) return launch_d<128, false, true>(tq, tk, tv, p, stream);
-  return launch_d<64, false, true>(tq, tk, tv, p, stream);
+  const FwdParams p = make_params(out, static_cast<int32_t>(bh), heads, g, s, scale, err_flag, limit_ns);
+  if (d == 128) return launch_d<128, false, kRaster>(tq, tk, tv, p, stream);
+  return launch_d<64, false, kRaster>(tq, tk, tv, p, stream);
+}
+
+cudaError_t launch_attention_mixed(const void* q, const void* k_tiled, const void* v_tiled, void* out, int32_t batch,
+                                   int32_t heads, int32_t d, const Geometry& g, const DeviceSchedule& s, float scale,
+                                   int32_t* err_flag, uint64_t limit_ns, cudaStream_t stream) {
+  if (s.masked || !raster_tile_ok(g.tt, g.th, g.tw) || g.ntile % kBlockRows != 0) return cudaErrorInvalidValue;
+  const int64_t bh = static_cast<int64_t>(batch) * heads;
+  const int bt = kBlockRows / (g.th * g.tw);
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap_raster(&tq, q, bh, g, d, bt) || !make_tmap(&tk, k_tiled, bh, g.Lpad, d) ||
+      !make_tmap(&tv, v_tiled, bh, g.Lpad, d))
+    return cudaErrorInvalidValue;
+  const FwdParams p = make_params(out, static_cast<int32_t>(bh), heads, g, s, scale, err_flag, limit_ns);
+  if (d == 128) return launch_d<128, false, kMixed>(tq, tk, tv, p, stream);
+  return launch_d<64, false, kMixed>(tq, tk, tv, p, stream);
 }
 
 cudaError_t launch_selftest_wait(int32_t* err_flag, uint64_t limit_ns, cudaStream_t stream) {

@@ -93,6 +93,11 @@ cudaError_t launch_reorder(const void* src, void* dst, int64_t batch_heads, int3
                            const Geometry& g, bool to_tiled, cudaStream_t stream,
                            int32_t token_major_heads = 0);
 
+// Raster [BH, T*H*W, d] -> tiled order of the padded latent [BH, Lpad, d], the
+// rows of pad tokens written as zeros (reorder.cu).
+cudaError_t launch_reorder_padded(const void* src, void* dst, int64_t batch_heads, int32_t d, const Geometry& g,
+                                  cudaStream_t stream);
+
 struct DeviceSchedule {
   const WorkItem* items;
   const int32_t* kv_rows;
@@ -101,6 +106,8 @@ struct DeviceSchedule {
   bool masked;
   const int32_t* kv_mask_id = nullptr;   // padded latents only
   const uint32_t* kv_masks = nullptr;
+  int32_t n_kv_rows = 0;                 // entries of kv_rows (for the device checks)
+  int32_t n_masks = 0;                   // 128-bit masks in kv_masks
 };
 
 // Attention on tiled-order tensors ([BH, L, d]); lse, when not null, receives
@@ -116,6 +123,14 @@ cudaError_t launch_attention_raster(const void* q, const void* k, const void* v,
                                     int32_t batch, int32_t heads, int32_t d, const Geometry& g,
                                     const DeviceSchedule& s, float scale, int32_t* err_flag,
                                     uint64_t limit_ns, cudaStream_t stream);
+
+// Attention with raster-order q and out ([BH, T, H, W, d], as the raster launcher)
+// and k, v in the tiled order of the padded latent ([BH, Lpad, d], pad rows zero,
+// as launch_reorder_padded writes them).
+cudaError_t launch_attention_mixed(const void* q, const void* k_tiled, const void* v_tiled, void* out,
+                                   int32_t batch, int32_t heads, int32_t d, const Geometry& g,
+                                   const DeviceSchedule& s, float scale, int32_t* err_flag,
+                                   uint64_t limit_ns, cudaStream_t stream);
 
 // Backward pass on tiled-order tensors: D = rowsum(dout * out) into dvec ([BH, L]
 // fp32 scratch), then dq over the forward schedule and dk, dv over the transposed

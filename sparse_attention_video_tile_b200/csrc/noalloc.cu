@@ -167,6 +167,7 @@ extern "C" sta_status sta_attention_fwd_noalloc(const void* q, const void* k, co
                     reinterpret_cast<const int32_t*>(nd.base + nd.off_kv),
                     reinterpret_cast<const int16_t*>(nd.base + nd.off_win),
                     static_cast<int32_t>(nd.sched.items.size()), nd.sched.masked};
+  ds.n_kv_rows = static_cast<int32_t>(nd.sched.kv_rows.size());
   e = launch_attention(q, k, v, out, batch, heads, d, g, ds, scale, reinterpret_cast<int32_t*>(nd.base),
                        kNoAllocWaitLimitNs, st);
   return e == cudaSuccess ? STA_OK : cuda_fail(e);

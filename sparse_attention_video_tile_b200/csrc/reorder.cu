@@ -8,6 +8,10 @@
 // bytes on both sides.  A warp copies a run with 16-byte vector loads and
 // stores; index arithmetic happens once per run, not per element.
 //
+// Padded variant (raster -> tiled only): for a latent that is not a tile
+// multiple, the tiled side has the rows of the padded latent (the tile grid
+// rounded up), and the rows of pad tokens are written as zeros.
+//
 // Token-major variant: the raster side is [B, L, heads, d], the layout of a
 // [B, L, heads * d] projection in a video transformer, and the tiled side is
 // [B, heads, L, d].  A run is then tw token rows heads * d elements apart on
@@ -22,7 +26,7 @@ namespace sta {
 namespace {
 
 struct RunGeo {
-  int64_t n_runs;          // batch_heads * L / tw
+  int64_t n_runs;          // batch_heads * L / tw (padded: batch_heads * Lpad / tw)
   int32_t runs_per_bh;     // L / tw
   int32_t runs_per_tile;   // tt * th
   int32_t th, tw, tt;
@@ -31,6 +35,8 @@ struct RunGeo {
   int32_t ntile;
   int64_t L;
   int32_t heads;           // token-major only
+  int32_t T;               // padded only: grid
+  int64_t Lpad;            // padded only: rows of the tiled side per batch*head
 };
 
 __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
@@ -96,7 +102,80 @@ __global__ void __launch_bounds__(256, 6) reorder_kernel(const uint4* __restrict
   }
 }
 
+// Raster [BH, T*H*W, d] -> padded tiled [BH, Lpad, d], pad rows zero.  Same
+// runs as reorder_kernel over the padded tile grid; a run (tw tokens of one tile
+// row) reads only the tokens inside the grid.
+template <int CPR>
+__global__ void __launch_bounds__(256, 6) reorder_padded_kernel(const uint4* __restrict__ src,
+                                                             uint4* __restrict__ dst, RunGeo g) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const int chunks = g.tw * CPR;
+  for (int64_t r = warp0; r < g.n_runs; r += nwarps) {
+    const int64_t bh = r / g.runs_per_bh;
+    const int32_t rr = static_cast<int32_t>(r - bh * g.runs_per_bh);
+    const int32_t tile_id = rr / g.runs_per_tile;
+    const int32_t rem = rr - tile_id * g.runs_per_tile;
+    const int32_t lt = rem / g.th;
+    const int32_t lh = rem - lt * g.th;
+    const int32_t at = tile_id / (g.nH * g.nW);
+    const int32_t ah = (tile_id / g.nW) % g.nH;
+    const int32_t aw = tile_id % g.nW;
+    const int64_t tiled_row = bh * g.Lpad + static_cast<int64_t>(tile_id) * g.ntile + (lt * g.th + lh) * g.tw;
+    const int32_t t = at * g.tt + lt, h = ah * g.th + lh, w0 = aw * g.tw;
+    // real tokens of the run: w0 .. w0 + real - 1
+    const int32_t real = (t < g.T && h < g.H) ? min(g.tw, max(g.W - w0, 0)) : 0;
+    const int64_t n0 = (static_cast<int64_t>(t) * g.H + h) * g.W + w0;
+    const uint4* sp = src + (bh * g.L + n0) * CPR;
+    uint4* dp = dst + tiled_row * CPR;
+    for (int base = 0; base < chunks; base += 4 * 32) {
+      uint4 buf[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = base + u * 32 + lane;
+        buf[u] = make_uint4(0u, 0u, 0u, 0u);
+        if (i < chunks && i / CPR < real) buf[u] = ld_stream(sp + i);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = base + u * 32 + lane;
+        if (i < chunks) dp[i] = buf[u];
+      }
+    }
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_reorder_padded(const void* src, void* dst, int64_t batch_heads, int32_t d, const Geometry& geo,
+                                  cudaStream_t stream) {
+  RunGeo g;
+  g.heads = 0;
+  g.runs_per_bh = static_cast<int32_t>(geo.Lpad / geo.tw);
+  g.n_runs = batch_heads * g.runs_per_bh;
+  g.runs_per_tile = geo.tt * geo.th;
+  g.th = geo.th; g.tw = geo.tw; g.tt = geo.tt;
+  g.nH = geo.nH; g.nW = geo.nW;
+  g.H = geo.H; g.W = geo.W; g.T = geo.T;
+  g.ntile = geo.ntile;
+  g.L = geo.L;
+  g.Lpad = geo.Lpad;
+  if (g.n_runs == 0) return cudaSuccess;
+  int dev = 0, sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  int64_t blocks = (g.n_runs + 7) / 8;
+  const int64_t max_blocks = static_cast<int64_t>(sms) * 8;
+  if (blocks > max_blocks) blocks = max_blocks;
+  const uint4* s = static_cast<const uint4*>(src);
+  uint4* dd = static_cast<uint4*>(dst);
+  if (d == 128) reorder_padded_kernel<16><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(s, dd, g);
+  else reorder_padded_kernel<8><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(s, dd, g);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_reorder(const void* src, void* dst, int64_t batch_heads, int32_t d,
                            const Geometry& geo, bool to_tiled, cudaStream_t stream, int32_t token_major_heads) {

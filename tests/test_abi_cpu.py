@@ -234,3 +234,38 @@ def test_schedules_cover_exactly_the_window_blocks(lib, name, cfg):
 def test_schedule_pairs_reject_small_tiles(lib):
     assert lib.sta_schedule_block_pairs(1, 1, sta._d3((4, 8, 8)), sta._d3((2, 4, 4)), sta._windows([(1, 1, 1)]),
                                         0, None, 0) == -1
+
+
+def _call_mixed(lib, q=0x1000000, kt=0x2000000, vt=0x3000000, out=0x4000000, batch=1, heads=1, d=128,
+                grid=(11, 22, 37), tile=(6, 8, 8), windows=((1, 3, 3),), scale=0.1):
+    return lib.sta_attention_fwd_mixed(q, kt, vt, out, batch, heads, d, sta._d3(grid), sta._d3(tile),
+                                       sta._windows(windows), ctypes.c_float(scale), None)
+
+
+def test_padded_reorder_and_mixed_validation_codes(lib):
+    # fake pointers, never dereferenced: validation fails before the device is touched.
+    # (11, 22, 37) pads to (12, 24, 40): 8954 raster rows, 11520 tiled rows.
+    A, B = 0x1000000, 0x2000000
+    pad = lambda src, dst, **kw: lib.sta_tile_reorder_padded(src, dst, kw.get("bh", 1), kw.get("d", 128),  # noqa: E731
+                                                             sta._d3(kw.get("grid", (11, 22, 37))),
+                                                             sta._d3(kw.get("tile", (6, 8, 8))), None)
+    assert pad(None, B) == 1
+    assert pad(A + 4, B) == 2
+    assert pad(A, A + 8954 * 256 - 16) == 3          # dst starts inside src
+    assert pad(A + 11520 * 256 - 16, A) == 3         # src starts inside the (larger) dst
+    assert pad(A, B, grid=(0, 22, 37)) == 4
+    assert pad(A, B, d=96) == 6
+    assert pad(A, B, bh=-1) == 10
+    assert _call_mixed(lib, q=None) == 1
+    assert _call_mixed(lib, vt=0x3000008) == 2
+    assert _call_mixed(lib, out=0x2000000 + 256 * 100) == 3     # out over k_tiled
+    assert _call_mixed(lib, tile=(2, 4, 4)) == 4                # 32-token tiles
+    assert _call_mixed(lib, tile=(1, 8, 12)) == 4               # not 128-row slabs of whole frames
+    assert _call_mixed(lib, windows=((1, 0, 3),)) == 5
+    assert _call_mixed(lib, d=48) == 6
+    assert _call_mixed(lib, scale=0.0) == 10
+    import torch
+    if not torch.cuda.is_available():
+        # valid arguments and no GPU: a CUDA/architecture error, never a host computation
+        assert pad(A, B) in (7, 8)
+        assert _call_mixed(lib) in (7, 8)

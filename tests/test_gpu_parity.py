@@ -154,6 +154,67 @@ def test_attention_padded_latents(cfg):
     _full_parity(cfg, seed=6, pad=True)
 
 
+def _padded_tiled_reference(x, grid, tile):
+    """The oracle's construction of the padded latent's tiled order: zero tokens
+    added up to tile multiples, then the tile map of that grid."""
+    T, H, Wd = grid
+    Tp, Hp, Wp = (-(-a // b) * b for a, b in zip(grid, tile))
+    lead = x.shape[:-2]
+    d = x.shape[-1]
+    full = torch.zeros(lead + (Tp, Hp, Wp, d), dtype=x.dtype, device=x.device)
+    full[..., :T, :H, :Wd, :] = x.reshape(lead + (T, H, Wd, d))
+    full = full.reshape(lead + (Tp * Hp * Wp, d))
+    m = torch.from_numpy(O.tiled_of_raster((Tp, Hp, Wp), tile)).to(x.device)
+    out = torch.empty_like(full)
+    out[..., m, :] = full
+    return out
+
+
+@pytest.mark.parametrize("cfg", PADDED + [W.CONFIGS["small"]], ids=lambda c: c.name)
+def test_padded_reorder_bit_exact(cfg):
+    g = torch.Generator(device="cuda").manual_seed(3)
+    x = torch.randn((cfg.batch, cfg.heads, cfg.L, cfg.d), device="cuda", generator=g).to(torch.bfloat16)
+    y = torch.full((cfg.batch, cfg.heads, sta.padded_rows(cfg.grid, cfg.tile), cfg.d), float("nan"),
+                   device="cuda", dtype=torch.bfloat16)
+    sta.sta_tile_reorder_padded(x, y, cfg.grid, cfg.tile)
+    assert torch.equal(y, _padded_tiled_reference(x, cfg.grid, cfg.tile))
+    if cfg.grid[0] % cfg.tile[0] == 0 and cfg.grid[1] % cfg.tile[1] == 0 and cfg.grid[2] % cfg.tile[2] == 0:
+        z = torch.empty_like(x)
+        sta.sta_tile_reorder(x, z, cfg.grid, cfg.tile)
+        assert torch.equal(y, z)
+    torch.cuda.synchronize()
+
+
+@pytest.mark.parametrize("cfg", PADDED, ids=lambda c: c.name)
+def test_mixed_path_padded_latents(cfg):
+    """Raster q and output, padded tiled k and v: every row against the oracle, and
+    bit for bit the one-launch raster path (same schedule and arithmetic)."""
+    q, k, v = W.make_qkv(cfg, 6)
+    qd, kd, vd = (x.cuda() for x in (q, k, v))
+    got = sta.sta_forward(qd, kd, vd, cfg.grid, cfg.tile, cfg.windows, cfg.scale, path="mixed")
+    ref = sta.sta_forward(qd, kd, vd, cfg.grid, cfg.tile, cfg.windows, cfg.scale, path="fused")
+    torch.cuda.synchronize()
+    assert sta.sta_check_device_status() == sta.STA_OK
+    assert torch.equal(got, ref)
+    out = got.float().cpu().numpy()
+    for b in range(cfg.batch):
+        for h in range(cfg.heads):
+            want = O.sta_attention_head(q[b, h].double().numpy(), k[b, h].double().numpy(), v[b, h].double().numpy(),
+                                        cfg.grid, cfg.tile, cfg.windows[h], cfg.scale, pad=True)
+            _compare(out[b, h], want, f"{cfg.name} mixed b{b} h{h}")
+
+
+@pytest.mark.parametrize("name", ["small", "image2d", "hunyuan"])
+def test_mixed_path_equals_three_call_path(name):
+    cfg = W.CONFIGS[name]
+    q, k, v = (x.cuda() for x in W.make_qkv(cfg, 2))
+    a = sta.sta_forward(q, k, v, cfg.grid, cfg.tile, cfg.windows, cfg.scale, path="mixed")
+    b = sta.sta_forward(q, k, v, cfg.grid, cfg.tile, cfg.windows, cfg.scale, path="three_call")
+    torch.cuda.synchronize()
+    assert sta.sta_check_device_status() == sta.STA_OK
+    assert torch.equal(a, b)
+
+
 LSE_ABS = 1e-3   # fp32 scores from bf16 inputs, MUFU exponentials, fp32 sums: about 1e-5 expected
 
 
