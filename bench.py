@@ -1,10 +1,12 @@
 """Benchmark of the Sliding Tile Attention forward path on B200.
 
-One step = the whole hot path on one batch of synthetic input: tile reorder of
-q, k and v, tile-windowed attention, reorder of the output back (five launches:
-reorder x3, tiled attention, unorder).  --fused times the one-launch fused
-raster-order kernel as the step instead; the other path is timed beside it and
-reported under `kernels`.  The default workload is the HunyuanVideo-shaped one
+One step = the whole hot path on one batch of synthetic input, raster-order q,
+k, v in, raster-order output out.  By default (--path mixed) that is the tile
+reorder of k and v into the padded latent's tiled order (two launches) and the
+attention kernel that reads q and writes the output in raster order (one
+launch).  --path three_call times reorder x3 + tiled attention + unorder (five
+launches), --path fused (or --fused) the one-launch raster-order kernel; the
+paths not timed as the step are timed beside it and reported under `kernels`.  The default workload is the HunyuanVideo-shaped one
 (latent 30x48x80 = 115200 tokens, tile (6,8,8), window (3,3,3) tiles, 24 heads,
 d = 128, bf16).
 
@@ -33,15 +35,16 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "STA fwd ms & TFLOPS (attended) at 30×48×80, 24 heads, d=128; % of BF16 peak"
-DEFAULT_PATH = "three_call"
+DEFAULT_PATH = "mixed"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM bytes (read + write) per launch of the tiled-order attention kernel on the default
 # workload, from an ncu capture of the 4-head case of that workload (scaled by 6 to 24 heads:
 # traffic is per head).  Valid only for the kernel source it was taken on, identified by the
 # SHA-1 of attention.cu and ptx.cuh.
-PROFILED_TRAFFIC = {"sha1": "841d955e9b881b000798eef7c4add12c8acca63c", "bytes_per_launch": 6 * (362.627072e6 + 106.815232e6),
-                    "workload": "hunyuan"}
+PROFILED_TRAFFIC = {"sha1": "86c7d06cacebada23b3d1ebbae2254a907c8779d", "workload": "hunyuan",
+                    "bytes_per_launch": {"mixed": 6 * (365.485056e6 + 103.638528e6),
+                                         "three_call": 6 * (363.680256e6 + 103.686400e6)}}
 
 
 def kernel_source_sha1():
@@ -477,7 +480,7 @@ def run_ours(args, cfg):
     att_tflops = flops / (att_ms * 1e-3) / 1e12
     traffic = None
     if cfg.name == PROFILED_TRAFFIC["workload"] and kernel_source_sha1() == PROFILED_TRAFFIC["sha1"]:
-        traffic = PROFILED_TRAFFIC["bytes_per_launch"]
+        traffic = PROFILED_TRAFFIC["bytes_per_launch"].get(args.path)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
