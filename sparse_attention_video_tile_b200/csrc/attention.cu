@@ -43,6 +43,9 @@
 //
 // Every barrier that is waited on with a parity can never run two phases ahead
 // of its waiter (the per-buffer S, P and P*V barriers, the Q pair, the ring).
+// The issuers wait for the loads that have almost always landed (K and Q for the
+// S issuer, V for the P*V issuer where that is safe) before the wait on the
+// S -> P -> P*V -> S chain, so that those checks are not on the chain.
 // With Ntile a multiple of 128 no element mask exists at all.  Otherwise (small
 // tiles, ragged tails) the softmax masks whole key tiles outside the row's
 // window and keys past L; padded latents mask the pad keys of boundary blocks.
@@ -377,8 +380,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int b = g % kSBufs;
           const int qb = c.k % S::kQBufs;
           const uint32_t seq = static_cast<uint32_t>(g + (g > 2 ? g - 2 : 0));
-          ok = (g < kSBufs || mbar_wait(sb + S::kPvDone + 8 * b, ((g / kSBufs) & 1) ^ 1, wc, 14)) &&
-               (c.j != 0 || mbar_wait(sb + S::kQFull + 8 * qb, (c.k / S::kQBufs) & 1, wc, 3)) && wait_load(seq, 4);
+          // K_g and Q first: they have almost always landed, and waiting for them while
+          // P V of block g-3 still runs keeps them off the S -> P -> P V -> S chain.  (The
+          // load before K_g on its stage is K_g-2, which this thread waited for itself.)
+          ok = wait_load(seq, 4) && (c.j != 0 || mbar_wait(sb + S::kQFull + 8 * qb, (c.k / S::kQBufs) & 1, wc, 3)) &&
+               (g < kSBufs || mbar_wait(sb + S::kPvDone + 8 * b, ((g / kSBufs) & 1) ^ 1, wc, 14));
           if (!ok) break;
           tc_fence_after();
           const uint32_t st = seq % kStages;
@@ -404,8 +410,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           // when g = 1) has landed and the parity wait for V_g cannot pass early.  An
           // item's first product (accumulate = 0) also waits until every softmax warp
           // has read the previous item's O.
-          ok = mbar_wait(sb + S::kPFull + 8 * b, (g / kSBufs) & 1, wc, 5) && wait_load(seq, 6) &&
-               (c.j != 0 || c.k == 0 || mbar_wait(sb + S::kOFree, static_cast<uint32_t>(c.k - 1) & 1, wc, 15));
+          // V_g before P_g only where the load before V_g on its stage is V_g-2, which this
+          // thread waited for itself (g >= 2 with V_g at ring load 2g + 3); elsewhere P_g
+          // first, which implies S_g ran and so every earlier load on the stage landed.
+          if (g >= 2 && seq == static_cast<uint32_t>(2 * g + 3))
+            ok = wait_load(seq, 6) && mbar_wait(sb + S::kPFull + 8 * b, (g / kSBufs) & 1, wc, 5);
+          else
+            ok = mbar_wait(sb + S::kPFull + 8 * b, (g / kSBufs) & 1, wc, 5) && wait_load(seq, 6);
+          ok = ok && (c.j != 0 || c.k == 0 || mbar_wait(sb + S::kOFree, static_cast<uint32_t>(c.k - 1) & 1, wc, 15));
           if (!ok) break;
           tc_fence_after();
           const uint32_t st = seq % kStages;

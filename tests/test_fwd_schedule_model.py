@@ -57,10 +57,11 @@ class Bar:
 
 class Forward:
     def __init__(self, items, seed, quads=2, stages=4, o_free=False, p_before_v=False, mutation=None,
-                 p_redo=0.25):
+                 p_redo=0.25, early_waits=False):
         self.rng = random.Random(seed)
         self.items, self.quads, self.stages = items, quads, stages
         self.o_free, self.p_before_v, self.mutation, self.p_redo = o_free, p_before_v, mutation, p_redo
+        self.early_waits = early_waits
         self.blocks = [(k, j) for k, n in enumerate(items) for j in range(n)]
         self.G = len(self.blocks)
         self.bars = {"OFull": Bar(1), "OFree": Bar(2 * quads)}
@@ -163,11 +164,17 @@ class Forward:
     def s_issuer(self):
         for g, (k, j) in enumerate(self.blocks):
             b, seq = g % 3, self.seq_k(g)
+            k_wait = self.wait(f"KvFull{seq % self.stages}", (seq // self.stages) & 1)
+            if self.early_waits:       # K (and Q) before the buffer: they are off the chain
+                yield k_wait
+                if j == 0:
+                    yield self.wait(f"QFull{k % 2}", (k // 2) & 1)
             if g >= 3 and self.mutation != "no_pvdone_wait":
                 yield self.wait(f"PvDone{b}", ((g // 3) & 1) ^ 1)
-            if j == 0:
-                yield self.wait(f"QFull{k % 2}", (k // 2) & 1)
-            yield self.wait(f"KvFull{seq % self.stages}", (seq // self.stages) & 1)
+            if not self.early_waits:
+                if j == 0:
+                    yield self.wait(f"QFull{k % 2}", (k // 2) & 1)
+                yield k_wait
             self.issue("S", g)
             self.commit("S", f"KvEmpty{seq % self.stages}")
             if j + 1 == self.items[k]:
@@ -179,7 +186,10 @@ class Forward:
             b, seq = g % 3, self.seq_v(g)
             v_wait = self.wait(f"KvFull{seq % self.stages}", (seq // self.stages) & 1)
             p_wait = self.wait(f"PFull{b}", (g // 3) & 1)
-            for w in ((p_wait, v_wait) if self.p_before_v else (v_wait, p_wait)):
+            # V first is safe once the stage's previous load is V_g-2, which this thread
+            # waited for itself (the steady part of the ring order, g >= 2)
+            v_first = not self.p_before_v or (self.early_waits and g >= 2 and seq == 2 * g + 3)
+            for w in ((v_wait, p_wait) if v_first else (p_wait, v_wait)):
                 yield w
             if self.o_free and j == 0 and k > 0:
                 yield self.wait("OFree", (k - 1) & 1)
@@ -283,8 +293,10 @@ def _failures(n, seed, **kw):
 
 
 def test_kernel_order_has_no_deadlock_and_no_stale_read():
-    # the order of csrc/attention.cu: O-free barrier, P_g before V_g
-    assert _failures(3000, 1, o_free=True, p_before_v=True) == []
+    # the order of csrc/attention.cu: O-free barrier, P_g before V_g except where V_g's stage
+    # last held V_g-2, and the S issuer's K and Q waits before its buffer wait
+    assert _failures(3000, 1, o_free=True, p_before_v=True, early_waits=True) == []
+    assert _failures(1000, 6, o_free=True, p_before_v=True) == []
 
 
 def test_without_the_two_orderings_the_model_finds_both_hazards():
@@ -300,5 +312,5 @@ def test_without_the_two_orderings_the_model_finds_both_hazards():
 
 @pytest.mark.parametrize("mutation", ["no_pvdone_wait", "no_outcome_read"])
 def test_model_catches_planted_ordering_mistakes(mutation):
-    fails = _failures(400, 4, o_free=True, p_before_v=True, mutation=mutation)
+    fails = _failures(400, 4, o_free=True, p_before_v=True, early_waits=True, mutation=mutation)
     assert len(fails) >= 40, f"{mutation}: caught in only {len(fails)} schedules"
