@@ -416,6 +416,8 @@ sta_status sta_attention_bwd(const void* q, const void* k, const void* v, const 
   if ((s = get_schedule(st, g, batch, heads, window_per_head, 0, &fw)) != STA_OK) return s;
   DeviceSchedule dfw{fw->d_items, fw->d_kv_rows, fw->d_head_win, static_cast<int32_t>(fw->host.items.size()), false};
   DeviceSchedule dtr{tr->d_items, tr->d_kv_rows, tr->d_head_win, static_cast<int32_t>(tr->host.items.size()), false};
+  dfw.n_kv_rows = static_cast<int32_t>(fw->host.kv_rows.size());
+  dtr.n_kv_rows = static_cast<int32_t>(tr->host.kv_rows.size());
   cudaError_t e = launch_backward(q, k, v, out, dout, lse, st->d_dvec, dq, dk, dv, batch, heads, d, g, dfw, dtr,
                                   scale, st->d_err, kWaitLimitNs, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? STA_OK : cuda_fail(e);

@@ -49,10 +49,20 @@
 #include "internal.h"
 #include "ptx.cuh"
 
+// Checked builds (STA_DEVICE_CHECKS=1) test every index taken from the work
+// schedule (items, streamed block rows) before it addresses memory, as in the
+// forward kernel: a failure records 0x200 | code, sets the abort flag and skips
+// the access.
+#ifndef STA_DEVICE_CHECKS
+#define STA_DEVICE_CHECKS 0
+#endif
+
 namespace sta {
 namespace {
 
 using namespace ptx;
+
+constexpr bool kBwdChecks = STA_DEVICE_CHECKS != 0;
 
 constexpr int kBwdThreads = 320;   // warps 0-7 elementwise + epilogue, 8 producer, 9 MMA issuer
 constexpr int kBwdProducer = 8;
@@ -74,6 +84,8 @@ struct BwdParams {
   float scale_log2;          // scale * log2(e)
   int32_t* err;
   uint64_t limit_ns;
+  int32_t n_rows;            // entries of rows (device checks)
+  int32_t n_bh;              // batch * heads (device checks)
 };
 
 template <int D>
@@ -184,6 +196,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int32_t idx = k * static_cast<int32_t>(gridDim.x) + static_cast<int32_t>(blockIdx.x);
         if (idx >= p.n_items) break;
         const WorkItem it = p.items[idx];
+        if (kBwdChecks && !(it.bh >= 0 && it.bh < p.n_bh && it.q_row0 >= 0 && it.q_row0 < p.L &&
+                            it.q_row0 % kBlockRows == 0 && it.kv_off >= 0 && it.kv_len >= 1 &&
+                            it.kv_off + it.kv_len <= p.n_rows)) {
+          atomicCAS(p.err, 0, 0x200 | 21);
+          *abort_flag = 1;
+          break;
+        }
         ok = mbar_wait(sb + S::kFixEmpty, (nfix & 1) ^ 1, wc, 1);
         if (!ok) break;
         ++nfix;
@@ -195,6 +214,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           ok = mbar_wait(sb + S::kKvEmpty + 8 * st, ((seq >> 1) & 1) ^ 1, wc, 2);
           if (!ok) break;
           const int32_t row = p.rows[it.kv_off + j];
+          if (kBwdChecks && !(row >= 0 && row < p.L && row % kBlockRows == 0)) {
+            atomicCAS(p.err, 0, 0x200 | 22);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
           const uint32_t base = sb + S::kStage0 + st * S::kStageBytes;
           const uint32_t full = sb + S::kKvFull + 8 * st;
           mbar_arrive_expect_tx(full, 2 * kBlockBytes + (KIND == kDkDv ? 1024u : 0u));
@@ -334,6 +359,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const int32_t idx = k * static_cast<int32_t>(gridDim.x) + static_cast<int32_t>(blockIdx.x);
       if (idx >= p.n_items) break;
       const WorkItem it = p.items[idx];
+      if (kBwdChecks && !(it.bh >= 0 && it.bh < p.n_bh && it.q_row0 >= 0 && it.q_row0 < p.L)) {
+        atomicCAS(p.err, 0, 0x200 | 23);
+        *abort_flag = 1;
+        break;
+      }
       const int64_t grow = static_cast<int64_t>(it.bh) * p.L + it.q_row0 + row;   // this thread's row
       float lse2_row = 0.f, d_row = 0.f;
       if (KIND == kDq) {
@@ -530,9 +560,11 @@ cudaError_t launch_backward(const void* q, const void* k, const void* v, const v
   p.scale_log2 = scale * 1.4426950408889634f;
   p.err = err_flag;
   p.limit_ns = limit_ns;
+  p.n_bh = static_cast<int32_t>(bh);
   // dQ over the forward's items
   p.items = fwd.items;
   p.rows = fwd.kv_rows;
+  p.n_rows = fwd.n_kv_rows;
   p.n_items = fwd.n_items;
   p.out0 = static_cast<__nv_bfloat16*>(dq);
   p.out1 = nullptr;
@@ -541,6 +573,7 @@ cudaError_t launch_backward(const void* q, const void* k, const void* v, const v
   // dK, dV over the transposed items
   p.items = tr.items;
   p.rows = tr.kv_rows;
+  p.n_rows = tr.n_kv_rows;
   p.n_items = tr.n_items;
   p.out0 = static_cast<__nv_bfloat16*>(dk);
   p.out1 = static_cast<__nv_bfloat16*>(dv);

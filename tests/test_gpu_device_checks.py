@@ -34,9 +34,28 @@ def _load(path):
         fn = getattr(lib, name)
         fn.restype = ctypes.c_int
         fn.argtypes = [P, P, P, P, I32, I32, I32, D3, D3, ctypes.POINTER(D3), F, P]
+    lib.sta_attention_fwd_lse.restype = ctypes.c_int
+    lib.sta_attention_fwd_lse.argtypes = [P, P, P, P, P, I32, I32, I32, D3, D3, ctypes.POINTER(D3), F, P]
+    lib.sta_attention_bwd.restype = ctypes.c_int
+    lib.sta_attention_bwd.argtypes = [P, P, P, P, P, P, P, P, P, I32, I32, I32, D3, D3, ctypes.POINTER(D3), F, P]
     lib.sta_check_device_status.restype = ctypes.c_int
     lib.sta_check_device_status.argtypes = [P]
     return lib
+
+
+def _backward(lib, cfg, q, k, v, do):
+    """Forward with log-sum-exp and backward through `lib` on tiled tensors."""
+    B, Hn, L, d = q.shape
+    s = torch.cuda.current_stream().cuda_stream
+    out = torch.empty_like(q)
+    lse = torch.empty((B, Hn, L), device=q.device, dtype=torch.float32)
+    g3, t3, w = sta._d3(cfg.grid), sta._d3(cfg.tile), sta._windows(cfg.windows)
+    assert lib.sta_attention_fwd_lse(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, Hn, d,
+                                     g3, t3, w, ctypes.c_float(cfg.scale), s) == 0
+    grads = [torch.full_like(q, float("nan")) for _ in range(3)]
+    assert lib.sta_attention_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), do.data_ptr(), lse.data_ptr(),
+                                 *(g.data_ptr() for g in grads), B, Hn, d, g3, t3, w, ctypes.c_float(cfg.scale), s) == 0
+    return grads
 
 
 @pytest.fixture(scope="module")
@@ -93,6 +112,18 @@ def test_checked_build_passes_and_matches_production(checked, path, cfg):
     assert torch.equal(got, want)
 
 
+def test_checked_build_backward_matches_production(checked):
+    cfg = W.custom_config("bwd_checked", 2, 3, 64, (4, 16, 24), (2, 8, 8), [(1, 1, 1), (3, 3, 3), (1, 2, 3)])
+    q, k, v = (x.cuda() for x in W.make_qkv(cfg, 5))
+    do = W.make_qkv(cfg, 105)[0].cuda()
+    got = _backward(checked, cfg, q, k, v, do)
+    assert checked.sta_check_device_status(ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)) == 0
+    want = _backward(sta.load_library(), cfg, q, k, v, do)
+    torch.cuda.synchronize()
+    for a, b in zip(got, want):
+        assert torch.equal(a, b)
+
+
 PLANT = r"""
 import ctypes, os, sys, torch
 sys.path.insert(0, ROOT)
@@ -100,7 +131,7 @@ sys.path.insert(0, HERE)
 import workloads as W
 import sparse_attention_video_tile_b200 as sta
 from sparse_attention_video_tile_b200.build import LIB_CHECKED
-from test_gpu_device_checks import _load, _call
+from test_gpu_device_checks import _load, _call, _backward
 sta.load_library()
 lib = _load(LIB_CHECKED)
 s = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
@@ -109,6 +140,11 @@ q, k, v = (x.cuda() for x in W.make_qkv(cfg, 1))
 out = torch.empty_like(q)
 assert _call(lib, "sta_attention_fwd", q, k, v, out, cfg) == 0     # schedule built with the planted row
 print("status", lib.sta_check_device_status(s))
+cfgb = W.custom_config("plant_bwd", 1, 2, 128, (6, 24, 24), (6, 8, 8), [(1, 3, 3), (1, 1, 1)])
+q, k, v = (x.cuda() for x in W.make_qkv(cfgb, 2))
+do = W.make_qkv(cfgb, 3)[0].cuda()
+_backward(lib, cfgb, q, k, v, do)             # the forward and the transposed schedules carry the planted row
+print("bwd", lib.sta_check_device_status(s))
 os.environ.pop("STA_CHECKS_PLANT_BAD_ROW")
 cfg2 = W.custom_config("clean", 1, 2, 128, (6, 24, 40), (6, 8, 8), [(1, 3, 3), (1, 1, 1)])
 q, k, v = (x.cuda() for x in W.make_qkv(cfg2, 1))
@@ -125,4 +161,5 @@ def test_checked_build_catches_a_planted_bad_row(checked):
     assert r.returncode == 0, r.stdout + r.stderr
     lines = dict(l.split(" ", 1) for l in r.stdout.strip().splitlines() if " " in l)
     assert lines["status"].strip() == str(STA_ERR_BOUNDS), r.stdout
+    assert lines["bwd"].strip() == str(STA_ERR_BOUNDS), r.stdout
     assert lines["after"].strip() == "0 True", r.stdout
