@@ -42,9 +42,9 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # workload, from an ncu capture of the 4-head case of that workload (scaled by 6 to 24 heads:
 # traffic is per head).  Valid only for the kernel source it was taken on, identified by the
 # SHA-1 of attention.cu and ptx.cuh.
-PROFILED_TRAFFIC = {"sha1": "86c7d06cacebada23b3d1ebbae2254a907c8779d", "workload": "hunyuan",
-                    "bytes_per_launch": {"mixed": 6 * (365.485056e6 + 103.638528e6),
-                                         "three_call": 6 * (363.680256e6 + 103.686400e6)}}
+PROFILED_TRAFFIC = {"sha1": "dde7cff513449cc04cb99a487486e9f846289de0", "workload": "hunyuan",
+                    "bytes_per_launch": {"mixed": 6 * (358.832896e6 + 103.412224e6),
+                                         "three_call": 6 * (359.112448e6 + 103.264256e6)}}
 
 
 def kernel_source_sha1():
