@@ -24,18 +24,24 @@
 //     dV += P^T dO and dK += dS^T Q; accumulators in columns 256-511);
 //   * warps 0-7 do the elementwise step in two phases: TMEM lane = row, warps w
 //     and w+4 take columns 0-63 and 64-127 of the rows of lane quadrant w.  Phase
-//     A turns S into P (fp32, in registers; for dK, dV also stored as bf16 P^T over
-//     S) and releases the S columns; phase B turns dP into dS and stores it as bf16
-//     over dP.  Each warp writes over the first 32 of its own 64 columns, so it never
-//     overwrites columns the other warp still reads.  At the end of an item each
-//     warp scales and stores its half of the accumulators' columns.
+//     A loads S, releases the S columns at once and turns S into P (fp32, in
+//     registers); phase B turns dP into dS and stores bf16 over the dP columns: dS
+//     over the first 32 of the warp's 64 columns (dQ), or P^T and dS^T interleaved
+//     over all 64 (dK, dV: per 32 columns, 16 of P^T then 16 of dS^T, each written
+//     after those 32 columns were read).  A warp never writes columns the other
+//     warp reads.  At the end of an item each warp scales and stores its half of
+//     the accumulators' columns.
 //
 // The two phases let the tensor core run beside the elementwise step: the issuer
-// starts the next block's S as soon as phase A has released the S columns, and the
-// accumulation and the next block's dP as soon as phase B has stored dS, so per
-// block the S product overlaps phase B and the accumulation plus dP overlap the
-// next block's phase A.  Two MMAs that touch the same TMEM columns (the next S over
-// P^T, the next dP over dS) come from the same thread and execute in issue order.
+// starts the next block's S as soon as phase A has loaded S, and the accumulations
+// and the next block's dP as soon as phase B has stored dS (and P^T), so the next
+// block's exponentials overlap this block's accumulations.  Two MMAs that touch the
+// same TMEM columns (the next dP over dS and P^T) come from the same thread and
+// execute in issue order.  The issuer's waits that have usually completed by the
+// time it reaches them (the next block's loads, the S of a block loaded, dS
+// stored) are tested without waiting in the middle of the MMA group before them,
+// so that their latency overlaps queued MMAs; a test that fails is followed by the
+// bounded wait at the point of use.
 //
 // Tiles must be multiples of 128 rows, so every block pair in a schedule is fully
 // attended and no mask exists.  Every wait is bounded (see ptx.cuh).
@@ -63,6 +69,19 @@ namespace {
 using namespace ptx;
 
 constexpr bool kBwdChecks = STA_DEVICE_CHECKS != 0;
+
+// True if the phase with parity `parity` of `bar` has completed; never waits.
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
 
 constexpr int kBwdThreads = 320;   // warps 0-7 elementwise + epilogue, 8 producer, 9 MMA issuer
 constexpr int kBwdProducer = 8;
@@ -102,8 +121,8 @@ struct BwdSmem {
   static constexpr int kKvEmpty = kKvFull + 16;    // [2]
   static constexpr int kSFull = kKvEmpty + 16;    // S (S^T) of a block in TMEM
   static constexpr int kDFull = kSFull + 8;       // dP (dP^T) of a block in TMEM
-  static constexpr int kSFree = kDFull + 8;       // phase A done: S read (dQ), P^T stored (dK, dV)
-  static constexpr int kPFull = kSFree + 8;       // phase B done: dS (dS^T) stored over dP
+  static constexpr int kSFree = kDFull + 8;       // phase A has loaded S (S^T)
+  static constexpr int kPFull = kSFree + 8;       // phase B done: dS (P^T and dS^T) stored over dP
   static constexpr int kOFull = kPFull + 8;
   static constexpr int kDrain = kOFull + 8;
   static constexpr int kTmemSlot = kDrain + 8;
@@ -243,11 +262,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   } else if (warp == kBwdMma) {
     if (lane == 0) {
       // Issue order per block b of the CTA's stream (stage b & 1):
-      //   wait phase A of b -> [dK, dV: dV += P^T dO] -> S of b+1 (within an item)
-      //   -> wait phase B of b -> dQ += dS K (or dK += dS^T Q) -> release the stage
+      //   wait S of b loaded -> S of b+1 (within an item) -> wait phase B of b
+      //   -> dQ += dS K (or dV += P^T dO, dK += dS^T Q) -> release the stage
       //   -> [item boundary: wait the next fixed operands, S of b+1] -> dP of b+1.
       // One thread issues everything, so a later MMA that overwrites an operand an
-      // earlier one reads (S over P^T, dP over dS) executes after it.
+      // earlier one reads (dP over dS and P^T) executes after it.
       constexpr uint32_t idesc_ss = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t idesc_ts = idesc_bf16_f32(128, D, false, true);
       const uint64_t dfix0 = sdesc_sw128(sb + S::kFix0, 16, 1024);
@@ -255,16 +274,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       auto koff = [](int k16) -> uint64_t { return static_cast<uint64_t>(((k16 >> 2) * 16384 + (k16 & 3) * 32) >> 4); };
       const uint32_t tS = tmem, tP = tmem + 128, tA0 = tmem + 256, tA1 = tmem + 384;
       auto stage_base = [&](uint32_t b) { return sb + S::kStage0 + (b & 1) * S::kStageBytes; };
-      auto issue_s = [&](uint32_t b) {   // S (S^T) = fix0 str0^T, K-major operands
+      // `mid` runs after the first half of a group's MMAs (the early tests)
+      auto issue_s = [&](uint32_t b, auto&& mid) {   // S (S^T) = fix0 str0^T, K-major operands
         const uint64_t ds0 = sdesc_sw128(stage_base(b), 16, 1024);
 #pragma unroll
-        for (int k16 = 0; k16 < D / 16; ++k16) umma_ss(tS, dfix0 + koff(k16), ds0 + koff(k16), idesc_ss, k16 > 0);
+        for (int k16 = 0; k16 < D / 16; ++k16) {
+          if (k16 == D / 32) mid();
+          umma_ss(tS, dfix0 + koff(k16), ds0 + koff(k16), idesc_ss, k16 > 0);
+        }
         umma_commit(sb + S::kSFull);
       };
-      auto issue_dp = [&](uint32_t b) {  // dP (dP^T) = fix1 str1^T
+      auto issue_dp = [&](uint32_t b, auto&& mid) {  // dP (dP^T) = fix1 str1^T
         const uint64_t ds1 = sdesc_sw128(stage_base(b) + kBlockBytes, 16, 1024);
 #pragma unroll
-        for (int k16 = 0; k16 < D / 16; ++k16) umma_ss(tP, dfix1 + koff(k16), ds1 + koff(k16), idesc_ss, k16 > 0);
+        for (int k16 = 0; k16 < D / 16; ++k16) {
+          if (k16 == D / 32) mid();
+          umma_ss(tP, dfix1 + koff(k16), ds1 + koff(k16), idesc_ss, k16 > 0);
+        }
         umma_commit(sb + S::kDFull);
       };
       auto item_len = [&](int32_t kk) -> int32_t {
@@ -272,16 +298,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         return idx < p.n_items ? p.items[idx].kv_len : 0;
       };
       auto kv_full = [&](uint32_t b) { return mbar_wait(sb + S::kKvFull + 8 * (b & 1), (b >> 1) & 1, wc, 4); };
+      auto kv_test = [&](uint32_t b) { return mbar_test(sb + S::kKvFull + 8 * (b & 1), (b >> 1) & 1); };
       int32_t k = 0, j = 0, n = item_len(0);
       uint32_t seq = 0, nfix = 0;
+      // early test results for the current block: its S loaded, the next block's loads
+      bool s_free_ok = false, kv_ok = false;
       bool ok = n > 0;
       if (ok) {
         ok = mbar_wait(sb + S::kFixFull, 0, wc, 3) && kv_full(0);
         nfix = 1;
         if (ok) {
           tc_fence_after();
-          issue_s(0);
-          issue_dp(0);
+          issue_s(0, [] {});
+          issue_dp(0, [&] {
+            s_free_ok = mbar_test(sb + S::kSFree, 0);
+            kv_ok = n > 1 && kv_test(1);
+          });
           if (n == 1) umma_commit(sb + S::kFixEmpty);
         }
       }
@@ -292,34 +324,39 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const bool next_is_last = new_item ? n_next == 1 : j + 2 == n;
         const uint32_t base = stage_base(seq);
         // accumulations: B operands are the stage's blocks read MN-major (16 rows = 2 KB
-        // per K16 slice); A is bf16 in TMEM, keys (or queries) 0-63 in columns 0-31 and
-        // 64-127 in columns 64-95 of its region
+        // per K16 slice); A is bf16 in TMEM over the dP columns
         const uint64_t dm0 = sdesc_sw128(base, kBlockRows * 128, 1024);
         const uint64_t dm1 = sdesc_sw128(base + kBlockBytes, kBlockRows * 128, 1024);
-        ok = mbar_wait(sb + S::kSFree, seq & 1, wc, 5);
+        if (!s_free_ok) ok = mbar_wait(sb + S::kSFree, seq & 1, wc, 5);
         if (!ok) break;
-        tc_fence_after();
-        if (KIND == kDkDv) {
-          // dV += P^T dO (P^T over the S^T columns)
-#pragma unroll
-          for (int k16 = 0; k16 < 8; ++k16)
-            umma_ts(tA0, tS + (k16 >> 2) * 64 + (k16 & 3) * 8, dm1 + static_cast<uint64_t>(k16 * (2048 >> 4)), idesc_ts,
-                    (j > 0 || k16 > 0));
-        }
+        bool p_ok = false;
         if (has_next && !new_item) {   // next block's S while the elementwise warps finish this one
-          ok = kv_full(seq + 1);
+          if (!kv_ok) ok = kv_full(seq + 1);
           if (!ok) break;
           tc_fence_after();
-          issue_s(seq + 1);
+          issue_s(seq + 1, [&] { p_ok = mbar_test(sb + S::kPFull, seq & 1); });
         }
-        ok = mbar_wait(sb + S::kPFull, seq & 1, wc, 7);
+        if (!p_ok) ok = mbar_wait(sb + S::kPFull, seq & 1, wc, 7);
         if (!ok) break;
         tc_fence_after();
-        // dQ += dS K, or dK += dS^T Q; dS (dS^T) over the dP (dP^T) columns
+        if (KIND == kDq) {
+          // dQ += dS K; dS over the first 32 of each warp's 64 dP columns
 #pragma unroll
-        for (int k16 = 0; k16 < 8; ++k16)
-          umma_ts(KIND == kDq ? tA0 : tA1, tP + (k16 >> 2) * 64 + (k16 & 3) * 8,
-                  dm0 + static_cast<uint64_t>(k16 * (2048 >> 4)), idesc_ts, (j > 0 || k16 > 0));
+          for (int k16 = 0; k16 < 8; ++k16)
+            umma_ts(tA0, tP + (k16 >> 2) * 64 + (k16 & 3) * 8, dm0 + static_cast<uint64_t>(k16 * (2048 >> 4)),
+                    idesc_ts, (j > 0 || k16 > 0));
+        } else {
+          // dV += P^T dO and dK += dS^T Q; K16 slice k16 (16 queries) of P^T at column
+          // 64 (k16 / 4) + 32 ((k16 / 2) mod 2) + 8 (k16 mod 2) of the dP region, dS^T 16 further
+#pragma unroll
+          for (int k16 = 0; k16 < 8; ++k16)
+            umma_ts(tA0, tP + (k16 >> 2) * 64 + ((k16 >> 1) & 1) * 32 + (k16 & 1) * 8,
+                    dm1 + static_cast<uint64_t>(k16 * (2048 >> 4)), idesc_ts, (j > 0 || k16 > 0));
+#pragma unroll
+          for (int k16 = 0; k16 < 8; ++k16)
+            umma_ts(tA1, tP + (k16 >> 2) * 64 + ((k16 >> 1) & 1) * 32 + 16 + (k16 & 1) * 8,
+                    dm0 + static_cast<uint64_t>(k16 * (2048 >> 4)), idesc_ts, (j > 0 || k16 > 0));
+        }
         umma_commit(sb + S::kKvEmpty + 8 * (seq & 1));
         if (new_item) umma_commit(sb + S::kOFull);
         if (!has_next) break;
@@ -328,9 +365,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           ++nfix;
           if (!ok) break;
           tc_fence_after();
-          issue_s(seq + 1);
+          issue_s(seq + 1, [] {});
         }
-        issue_dp(seq + 1);
+        // early tests for block seq + 1: its S loaded, and block seq + 2's loads when
+        // it belongs to the same item (its S is then issued in the next iteration)
+        issue_dp(seq + 1, [&] {
+          s_free_ok = mbar_test(sb + S::kSFree, (seq + 1) & 1);
+          kv_ok = !next_is_last && kv_test(seq + 2);
+        });
         if (next_is_last) umma_commit(sb + S::kFixEmpty);
         ++seq;
         if (new_item) {
@@ -385,7 +427,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const float4* col_d4 = col_lse4 + 32;
         // phase A: P (P^T) of this thread's row over this warp's 64 columns, kept in fp32
         float pf[64];
-        if (KIND == kDq) {
+        {
           uint32_t s_lo[32], s_hi[32];
           tmem_ld32(tS, s_lo);
           tmem_ld32(tS + 32, s_hi);
@@ -393,34 +435,27 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(sb + S::kSFree);   // S may be overwritten by the next block's
+          if (KIND == kDq) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            pf[i] = ex2_approx(fmaf(__uint_as_float(s_lo[i]), sl2, -lse2_row));
-            pf[32 + i] = ex2_approx(fmaf(__uint_as_float(s_hi[i]), sl2, -lse2_row));
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            uint32_t s32[32], pk[16];
-            tmem_ld32(tS + 32 * c, s32);
-            tmem_wait_ld();
+            for (int i = 0; i < 32; ++i) {
+              pf[i] = ex2_approx(fmaf(__uint_as_float(s_lo[i]), sl2, -lse2_row));
+              pf[32 + i] = ex2_approx(fmaf(__uint_as_float(s_hi[i]), sl2, -lse2_row));
+            }
+          } else {
 #pragma unroll
             for (int i = 0; i < 32; i += 4) {
-              const float4 lv = col_lse4[8 * c + i / 4];
+              const float4 lv = col_lse4[i / 4], hv = col_lse4[8 + i / 4];
               const float l2[4] = {lv.x * kLog2e, lv.y * kLog2e, lv.z * kLog2e, lv.w * kLog2e};
+              const float h2[4] = {hv.x * kLog2e, hv.y * kLog2e, hv.z * kLog2e, hv.w * kLog2e};
 #pragma unroll
-              for (int u = 0; u < 4; ++u) pf[32 * c + i + u] = ex2_approx(fmaf(__uint_as_float(s32[i + u]), sl2, -l2[u]));
-              pk[i >> 1] = pack_bf16x2(pf[32 * c + i], pf[32 * c + i + 1]);
-              pk[(i >> 1) + 1] = pack_bf16x2(pf[32 * c + i + 2], pf[32 * c + i + 3]);
+              for (int u = 0; u < 4; ++u) {
+                pf[i + u] = ex2_approx(fmaf(__uint_as_float(s_lo[i + u]), sl2, -l2[u]));
+                pf[32 + i + u] = ex2_approx(fmaf(__uint_as_float(s_hi[i + u]), sl2, -h2[u]));
+              }
             }
-            tmem_st16(tS + 16 * c, pk);   // P^T over the first 32 of this warp's S^T columns
           }
-          tmem_wait_st();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(sb + S::kSFree);
         }
-        // phase B: dS = P (dP - D), bf16 over the first 32 of this warp's dP columns
+        // phase B: dS = P (dP - D), bf16 over this warp's dP columns (and P^T for dK, dV)
         ok = __all_sync(0xffffffffu, mbar_wait(sb + S::kDFull, seq & 1, wc, 10));
         if (!ok) break;
         tc_fence_after();
@@ -444,7 +479,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             dk[i >> 1] = pack_bf16x2(dsv[0], dsv[1]);
             dk[(i >> 1) + 1] = pack_bf16x2(dsv[2], dsv[3]);
           }
-          tmem_st16(tP + 16 * c, dk);
+          if (KIND == kDq) {
+            tmem_st16(tP + 16 * c, dk);
+          } else {
+            // columns 32c .. 32c + 31 were read above: P^T over the first 16, dS^T over the next 16
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 32; i += 2) pk[i >> 1] = pack_bf16x2(pf[32 * c + i], pf[32 * c + i + 1]);
+            tmem_st16(tP + 32 * c, pk);
+            tmem_st16(tP + 32 * c + 16, dk);
+          }
         }
         tmem_wait_st();
         tc_fence_before();
