@@ -38,13 +38,13 @@ METRIC = "STA fwd ms & TFLOPS (attended) at 30×48×80, 24 heads, d=128; % of BF
 DEFAULT_PATH = "mixed"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-# DRAM bytes (read + write) per launch of the tiled-order attention kernel on the default
+# DRAM bytes (read + write) per launch of each forward path's attention kernel on the default
 # workload, from an ncu capture of the 4-head case of that workload (scaled by 6 to 24 heads:
 # traffic is per head).  Valid only for the kernel source it was taken on, identified by the
-# SHA-1 of attention.cu and ptx.cuh.
-PROFILED_TRAFFIC = {"sha1": "dde7cff513449cc04cb99a487486e9f846289de0", "workload": "hunyuan",
-                    "bytes_per_launch": {"mixed": 6 * (358.832896e6 + 103.412224e6),
-                                         "three_call": 6 * (359.112448e6 + 103.264256e6)}}
+# SHA-1 of attention.cu and ptx.cuh (an edit of comments alone carries the figures over).
+PROFILED_TRAFFIC = {"sha1": "aac283984a506d99de1e3f967e22364c5365eff1", "workload": "hunyuan",
+                    "bytes_per_launch": {"mixed": 6 * (358.576128e6 + 103.734016e6),
+                                         "three_call": 6 * (357.326336e6 + 103.657216e6)}}
 
 
 def kernel_source_sha1():

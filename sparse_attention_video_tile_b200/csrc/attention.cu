@@ -249,196 +249,204 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int kBoxes = D / 64;
   constexpr uint32_t kBlockBytes = S::kBlockBytes;
 
-  if (warp >= 8) setmaxnreg_dec<kRegsOther>();
-  if (warp == kProducerWarp) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      prefetch_tmap(&tm_q);
-      prefetch_tmap(&tm_k);
-      prefetch_tmap(&tm_v);
-      uint32_t kv_seq = 0, q_loads[2] = {0, 0};
-      bool ok = true;
-      // one 128-row block (Q into buffer `dst`, or K/V into the next ring stage);
-      // `raster`: the tensor is in raster order, read as 5-D boxes
-      auto tma_block = [&](uint32_t dst, const CUtensorMap* m, uint32_t full, int32_t row, int32_t bh, bool raster) {
-        if (raster) {
-          const SlabCoord c = slab_coord(p, row);
-          for (int b = 0; b < kBoxes; ++b) tma_load_5d(dst + b * kBoxBytes, m, full, b * 64, c.w, c.h, c.t, bh);
-        } else {
-          for (int b = 0; b < kBoxes; ++b) tma_load_3d(dst + b * kBoxBytes, m, full, b * 64, row, bh);
-        }
-      };
-      auto load_ring = [&](const CUtensorMap* m, int32_t row, int32_t bh) -> bool {
-        const uint32_t st = kv_seq % kStages;
-        if (!mbar_wait(sb + S::kKvEmpty + 8 * st, ((kv_seq / kStages) & 1) ^ 1, wc, 2)) return false;
-        const uint32_t full = sb + S::kKvFull + 8 * st;
-        mbar_arrive_expect_tx(full, kBlockBytes);
-        tma_block(sb + S::kStage0 + st * kBlockBytes, m, full, row, bh, LAYOUT == kRaster);
-        ++kv_seq;
-        return true;
-      };
-      // failed device check: record it and stop; the CTA drains as after an expired wait
-      auto fail = [&](int code) {
-        atomicCAS(p.err, 0, 0x200 | code);
-        *abort_flag = 1;
-      };
-      // row of key block j of the cursor's item, or -1 after a failed check
-      auto kv_row = [&](const BlockCursor& c, int code) -> int32_t {
-        const int32_t idx = c.it.kv_off + c.j;
-        if (kChecks && !(idx >= 0 && idx < p.n_kv_rows)) {
-          fail(code);
-          return -1;
-        }
-        const int32_t row = p.kv_rows[idx];
-        if (kChecks && !(row >= 0 && row < p.rows && row % kBlockRows == 0)) {
-          fail(code + 1);
-          return -1;
-        }
-        return row;
-      };
-      // K of block (k, j), preceded by the item's Q when j = 0
-      auto load_k = [&](const BlockCursor& c) -> bool {
-        if (kChecks && !(c.it.bh >= 0 && c.it.bh < p.n_bh && c.it.q_row0 >= 0 && c.it.q_row0 < p.rows &&
-                         c.it.q_row0 % kBlockRows == 0 && c.it.kv_len >= 1)) {
-          fail(1);
-          return false;
-        }
-        if (c.j == 0) {
-          const int qb = c.k % S::kQBufs;
-          if (!mbar_wait(sb + S::kQEmpty + 8 * qb, ((c.k / S::kQBufs) & 1) ^ 1, wc, 1)) return false;
-          mbar_arrive_expect_tx(sb + S::kQFull + 8 * qb, kBlockBytes);
-          tma_block(sb + S::kQ + qb * kBlockBytes, &tm_q, sb + S::kQFull + 8 * qb, c.it.q_row0, c.it.bh, LAYOUT != kTiled);
-          ++q_loads[qb];
-        }
-        const int32_t row = kv_row(c, 2);
-        return row >= 0 && load_ring(&tm_k, row, c.it.bh);
-      };
-      // Order of the loads: K_0, K_1, K_2, then V_g, K_g+3 for g = 0, 1, ... (the S
-      // issuer needs K three blocks ahead of the P V issuer's V).
-      BlockCursor kc, vc;
-      kc.start(p);
-      vc.start(p);
-      for (int i = 0; i < kSBufs && ok && !kc.done; ++i) {
-        ok = load_k(kc);
-        kc.next(p);
-      }
-      while (ok && !vc.done) {
-        const int32_t row = kv_row(vc, 4);
-        ok = row >= 0 && load_ring(&tm_v, row, vc.it.bh);
-        vc.next(p);
-        if (ok && !kc.done) {
+  // The two role branches, softmax warps and the rest, as lambdas, so that the order in
+  // which they are placed in the code can be chosen per layout (end of the kernel).
+  auto other_roles = [&]() {
+    setmaxnreg_dec<kRegsOther>();
+    if (warp == kProducerWarp) {
+      // ------------------------------------------------------------ producer
+      if (lane == 0) {
+        prefetch_tmap(&tm_q);
+        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_v);
+        uint32_t kv_seq = 0, q_loads[2] = {0, 0};
+        bool ok = true;
+        // one 128-row block (Q into buffer `dst`, or K/V into the next ring stage);
+        // `raster`: the tensor is in raster order, read as 5-D boxes
+        auto tma_block = [&](uint32_t dst, const CUtensorMap* m, uint32_t full, int32_t row, int32_t bh, bool raster) {
+          if (raster) {
+            const SlabCoord c = slab_coord(p, row);
+            for (int b = 0; b < kBoxes; ++b) tma_load_5d(dst + b * kBoxBytes, m, full, b * 64, c.w, c.h, c.t, bh);
+          } else {
+            for (int b = 0; b < kBoxes; ++b) tma_load_3d(dst + b * kBoxBytes, m, full, b * 64, row, bh);
+          }
+        };
+        auto load_ring = [&](const CUtensorMap* m, int32_t row, int32_t bh) -> bool {
+          const uint32_t st = kv_seq % kStages;
+          if (!mbar_wait(sb + S::kKvEmpty + 8 * st, ((kv_seq / kStages) & 1) ^ 1, wc, 2)) return false;
+          const uint32_t full = sb + S::kKvFull + 8 * st;
+          mbar_arrive_expect_tx(full, kBlockBytes);
+          tma_block(sb + S::kStage0 + st * kBlockBytes, m, full, row, bh, LAYOUT == kRaster);
+          ++kv_seq;
+          return true;
+        };
+        // failed device check: record it and stop; the CTA drains as after an expired wait
+        auto fail = [&](int code) {
+          atomicCAS(p.err, 0, 0x200 | code);
+          *abort_flag = 1;
+        };
+        // row of key block j of the cursor's item, or -1 after a failed check
+        auto kv_row = [&](const BlockCursor& c, int code) -> int32_t {
+          const int32_t idx = c.it.kv_off + c.j;
+          if (kChecks && !(idx >= 0 && idx < p.n_kv_rows)) {
+            fail(code);
+            return -1;
+          }
+          const int32_t row = p.kv_rows[idx];
+          if (kChecks && !(row >= 0 && row < p.rows && row % kBlockRows == 0)) {
+            fail(code + 1);
+            return -1;
+          }
+          return row;
+        };
+        // K of block (k, j), preceded by the item's Q when j = 0
+        auto load_k = [&](const BlockCursor& c) -> bool {
+          if (kChecks && !(c.it.bh >= 0 && c.it.bh < p.n_bh && c.it.q_row0 >= 0 && c.it.q_row0 < p.rows &&
+                           c.it.q_row0 % kBlockRows == 0 && c.it.kv_len >= 1)) {
+            fail(1);
+            return false;
+          }
+          if (c.j == 0) {
+            const int qb = c.k % S::kQBufs;
+            if (!mbar_wait(sb + S::kQEmpty + 8 * qb, ((c.k / S::kQBufs) & 1) ^ 1, wc, 1)) return false;
+            mbar_arrive_expect_tx(sb + S::kQFull + 8 * qb, kBlockBytes);
+            tma_block(sb + S::kQ + qb * kBlockBytes, &tm_q, sb + S::kQFull + 8 * qb, c.it.q_row0, c.it.bh,
+                      LAYOUT != kTiled);
+            ++q_loads[qb];
+          }
+          const int32_t row = kv_row(c, 2);
+          return row >= 0 && load_ring(&tm_k, row, c.it.bh);
+        };
+        // Order of the loads: K_0, K_1, K_2, then V_g, K_g+3 for g = 0, 1, ... (the S
+        // issuer needs K three blocks ahead of the P V issuer's V).
+        BlockCursor kc, vc;
+        kc.start(p);
+        vc.start(p);
+        for (int i = 0; i < kSBufs && ok && !kc.done; ++i) {
           ok = load_k(kc);
           kc.next(p);
         }
-      }
-      // Drain: every load issued has landed before the CTA may exit.  Waiting on a
-      // phase that already completed returns at once.
-      for (int b = 0; b < S::kQBufs; ++b)
-        if (q_loads[b] > 0) mbar_wait_drain(sb + S::kQFull + 8 * b, (q_loads[b] - 1) & 1, p.limit_ns);
-      for (uint32_t s = 0; s < kStages && s < kv_seq; ++s) {
-        const uint32_t last = kv_seq - 1 - ((kv_seq - 1 - s) % kStages);  // last sequence number on stage s
-        mbar_wait_drain(sb + S::kKvFull + 8 * s, (last / kStages) & 1, p.limit_ns);
-      }
-    }
-    __syncwarp();
-  } else if (warp == kPvWarp || warp == kSWarp) {
-    // ------------------------------------------------------------ MMA issuers
-    // A tcgen05.mma issue returns at about the rate the tensor core executes, so
-    // whatever else an issuing thread does (barrier waits, commits, bookkeeping)
-    // leaves the tensor core idle unless another thread is issuing meanwhile: S
-    // and P*V have one issuer each.
-    if (lane == 0) {
-      // Shared-memory descriptors differ only in the start-address field (bits 0-13,
-      // address >> 4; every address here is below 256 KB, so adding an offset never
-      // carries out of the field): one base descriptor per role plus offsets.
-      constexpr uint32_t kBlockStep = kBlockBytes >> 4;
-      // Ring sequence numbers of the loads, in the producer's order K_0, K_1, K_2,
-      // V_0, K_3, V_1, ...: K_g is load g + max(0, g - 2) and V_g is load
-      // min(G + g, 2 g + 3), G being the number of blocks of this CTA.
-      int32_t G = 0;
-      for (int32_t k = 0;; ++k) {
-        const int32_t idx = k * static_cast<int32_t>(gridDim.x) + static_cast<int32_t>(blockIdx.x);
-        if (idx >= p.n_items) break;
-        G += p.items[idx].kv_len;
-      }
-      auto wait_load = [&](uint32_t seq, int site) -> bool {
-        return mbar_wait(sb + S::kKvFull + 8 * (seq % kStages), (seq / kStages) & 1, wc, site);
-      };
-      BlockCursor c;
-      c.start(p);
-      bool ok = true;
-      if (warp == kSWarp) {
-        // S_g = Q K_g^T into S buffer g mod 3, once P_g-3 V_g-3 (which reads P_g-3
-        // from that buffer) has completed.
-        constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
-        const uint64_t dq0 = sdesc_sw128(sb + S::kQ, 16, 1024);                         // K-major (Q)
-        const uint64_t dk0 = sdesc_sw128(sb + S::kStage0, 16, 1024);                    // K-major (K)
-        // slice k16 of a K-major block: 64-column boxes of 16 KB, 32 bytes per 16 columns
-        auto koff = [](int k16) -> uint64_t { return static_cast<uint64_t>(((k16 >> 2) * 16384 + (k16 & 3) * 32) >> 4); };
-        for (; ok && !c.done; c.next(p)) {
-          const int32_t g = c.g;
-          const int b = g % kSBufs;
-          const int qb = c.k % S::kQBufs;
-          const uint32_t seq = static_cast<uint32_t>(g + (g > 2 ? g - 2 : 0));
-          // K_g and Q first: they have almost always landed, and waiting for them while
-          // P V of block g-3 still runs keeps them off the S -> P -> P V -> S chain.  (The
-          // load before K_g on its stage is K_g-2, which this thread waited for itself.)
-          ok = wait_load(seq, 4) && (c.j != 0 || mbar_wait(sb + S::kQFull + 8 * qb, (c.k / S::kQBufs) & 1, wc, 3)) &&
-               (g < kSBufs || mbar_wait(sb + S::kPvDone + 8 * b, ((g / kSBufs) & 1) ^ 1, wc, 14));
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t st = seq % kStages;
-          const uint64_t dq = dq0 + qb * kBlockStep, dk = dk0 + st * kBlockStep;
-#pragma unroll
-          for (int k16 = 0; k16 < D / 16; ++k16)
-            umma_ss(tmem + 128 * b, dq + koff(k16), dk + koff(k16), idesc_qk, k16 > 0 ? 1u : 0u);
-          umma_commit(sb + S::kKvEmpty + 8 * st);
-          if (c.j + 1 == c.it.kv_len) umma_commit(sb + S::kQEmpty + 8 * qb);
-          umma_commit(sb + S::kSFull + 8 * b);
+        while (ok && !vc.done) {
+          const int32_t row = kv_row(vc, 4);
+          ok = row >= 0 && load_ring(&tm_v, row, vc.it.bh);
+          vc.next(p);
+          if (ok && !kc.done) {
+            ok = load_k(kc);
+            kc.next(p);
+          }
         }
-      } else {
-        // O += P_g V_g: keys 0-63 with P in S columns 0-31, keys 64-127 with P in
-        // S columns 64-95 (16 keys = 8 columns of P, 2 KB of V per slice)
-        constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
-        const uint32_t tO = tmem + kOCol;
-        const uint64_t dv0 = sdesc_sw128(sb + S::kStage0, kBlockRows * 128, 1024);      // MN-major (V)
-        for (; ok && !c.done; c.next(p)) {
-          const int32_t g = c.g;
-          const int b = g % kSBufs;
-          const uint32_t seq = static_cast<uint32_t>(min(G + g, 2 * g + 3));
-          // P_g first: it implies S_g ran, so K_g (the load before V_g on a ring stage
-          // when g = 1) has landed and the parity wait for V_g cannot pass early.  An
-          // item's first product (accumulate = 0) also waits until every softmax warp
-          // has read the previous item's O.
-          // V_g before P_g only where the load before V_g on its stage is V_g-2, which this
-          // thread waited for itself (g >= 2 with V_g at ring load 2g + 3); elsewhere P_g
-          // first, which implies S_g ran and so every earlier load on the stage landed.
-          if (g >= 2 && seq == static_cast<uint32_t>(2 * g + 3))
-            ok = wait_load(seq, 6) && mbar_wait(sb + S::kPFull + 8 * b, (g / kSBufs) & 1, wc, 5);
-          else
-            ok = mbar_wait(sb + S::kPFull + 8 * b, (g / kSBufs) & 1, wc, 5) && wait_load(seq, 6);
-          ok = ok && (c.j != 0 || c.k == 0 || mbar_wait(sb + S::kOFree, static_cast<uint32_t>(c.k - 1) & 1, wc, 15));
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t st = seq % kStages;
-          const uint64_t dv = dv0 + st * kBlockStep;
-          const uint32_t tP = tmem + 128 * b;
-#pragma unroll
-          for (int k16 = 0; k16 < 8; ++k16)
-            umma_ts(tO, tP + (k16 >> 2) * 64 + (k16 & 3) * 8, dv + static_cast<uint64_t>(k16 * (2048 >> 4)), idesc_pv,
-                    (c.j > 0 || k16 > 0) ? 1u : 0u);
-          umma_commit(sb + S::kKvEmpty + 8 * st);
-          umma_commit(sb + S::kPvDone + 8 * b);
-          if (c.j + 1 == c.it.kv_len) umma_commit(sb + S::kOFull);
+        // Drain: every load issued has landed before the CTA may exit.  Waiting on a
+        // phase that already completed returns at once.
+        for (int b = 0; b < S::kQBufs; ++b)
+          if (q_loads[b] > 0) mbar_wait_drain(sb + S::kQFull + 8 * b, (q_loads[b] - 1) & 1, p.limit_ns);
+        for (uint32_t s = 0; s < kStages && s < kv_seq; ++s) {
+          const uint32_t last = kv_seq - 1 - ((kv_seq - 1 - s) % kStages);  // last sequence number on stage s
+          mbar_wait_drain(sb + S::kKvFull + 8 * s, (last / kStages) & 1, p.limit_ns);
         }
       }
-      // Drain: all MMAs issued by this thread complete before TMEM is freed.
-      const uint32_t drain = sb + (warp == kSWarp ? S::kDrainS : S::kDrain);
-      umma_commit(drain);
-      mbar_wait_drain(drain, 0, p.limit_ns);
+      __syncwarp();
+    } else if (warp == kPvWarp || warp == kSWarp) {
+      // ------------------------------------------------------------ MMA issuers
+      // A tcgen05.mma issue returns at about the rate the tensor core executes, so
+      // whatever else an issuing thread does (barrier waits, commits, bookkeeping)
+      // leaves the tensor core idle unless another thread is issuing meanwhile: S
+      // and P*V have one issuer each.
+      if (lane == 0) {
+        // Shared-memory descriptors differ only in the start-address field (bits 0-13,
+        // address >> 4; every address here is below 256 KB, so adding an offset never
+        // carries out of the field): one base descriptor per role plus offsets.
+        constexpr uint32_t kBlockStep = kBlockBytes >> 4;
+        // Ring sequence numbers of the loads, in the producer's order K_0, K_1, K_2,
+        // V_0, K_3, V_1, ...: K_g is load g + max(0, g - 2) and V_g is load
+        // min(G + g, 2 g + 3), G being the number of blocks of this CTA.
+        int32_t G = 0;
+        for (int32_t k = 0;; ++k) {
+          const int32_t idx = k * static_cast<int32_t>(gridDim.x) + static_cast<int32_t>(blockIdx.x);
+          if (idx >= p.n_items) break;
+          G += p.items[idx].kv_len;
+        }
+        auto wait_load = [&](uint32_t seq, int site) -> bool {
+          return mbar_wait(sb + S::kKvFull + 8 * (seq % kStages), (seq / kStages) & 1, wc, site);
+        };
+        BlockCursor c;
+        c.start(p);
+        bool ok = true;
+        if (warp == kSWarp) {
+          // S_g = Q K_g^T into S buffer g mod 3, once P_g-3 V_g-3 (which reads P_g-3
+          // from that buffer) has completed.
+          constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
+          const uint64_t dq0 = sdesc_sw128(sb + S::kQ, 16, 1024);                         // K-major (Q)
+          const uint64_t dk0 = sdesc_sw128(sb + S::kStage0, 16, 1024);                    // K-major (K)
+          // slice k16 of a K-major block: 64-column boxes of 16 KB, 32 bytes per 16 columns
+          auto koff = [](int k16) -> uint64_t {
+            return static_cast<uint64_t>(((k16 >> 2) * 16384 + (k16 & 3) * 32) >> 4);
+          };
+          for (; ok && !c.done; c.next(p)) {
+            const int32_t g = c.g;
+            const int b = g % kSBufs;
+            const int qb = c.k % S::kQBufs;
+            const uint32_t seq = static_cast<uint32_t>(g + (g > 2 ? g - 2 : 0));
+            // K_g and Q first: they have almost always landed, and waiting for them while
+            // P V of block g-3 still runs keeps them off the S -> P -> P V -> S chain.  (The
+            // load before K_g on its stage is K_g-2, which this thread waited for itself.)
+            ok = wait_load(seq, 4) && (c.j != 0 || mbar_wait(sb + S::kQFull + 8 * qb, (c.k / S::kQBufs) & 1, wc, 3)) &&
+                 (g < kSBufs || mbar_wait(sb + S::kPvDone + 8 * b, ((g / kSBufs) & 1) ^ 1, wc, 14));
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t st = seq % kStages;
+            const uint64_t dq = dq0 + qb * kBlockStep, dk = dk0 + st * kBlockStep;
+  #pragma unroll
+            for (int k16 = 0; k16 < D / 16; ++k16)
+              umma_ss(tmem + 128 * b, dq + koff(k16), dk + koff(k16), idesc_qk, k16 > 0 ? 1u : 0u);
+            umma_commit(sb + S::kKvEmpty + 8 * st);
+            if (c.j + 1 == c.it.kv_len) umma_commit(sb + S::kQEmpty + 8 * qb);
+            umma_commit(sb + S::kSFull + 8 * b);
+          }
+        } else {
+          // O += P_g V_g: keys 0-63 with P in S columns 0-31, keys 64-127 with P in
+          // S columns 64-95 (16 keys = 8 columns of P, 2 KB of V per slice)
+          constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
+          const uint32_t tO = tmem + kOCol;
+          const uint64_t dv0 = sdesc_sw128(sb + S::kStage0, kBlockRows * 128, 1024);      // MN-major (V)
+          for (; ok && !c.done; c.next(p)) {
+            const int32_t g = c.g;
+            const int b = g % kSBufs;
+            const uint32_t seq = static_cast<uint32_t>(min(G + g, 2 * g + 3));
+            // P_g first: it implies S_g ran, so K_g (the load before V_g on a ring stage
+            // when g = 1) has landed and the parity wait for V_g cannot pass early.  An
+            // item's first product (accumulate = 0) also waits until every softmax warp
+            // has read the previous item's O.
+            // V_g before P_g only where the load before V_g on its stage is V_g-2, which this
+            // thread waited for itself (g >= 2 with V_g at ring load 2g + 3); elsewhere P_g
+            // first, which implies S_g ran and so every earlier load on the stage landed.
+            if (g >= 2 && seq == static_cast<uint32_t>(2 * g + 3))
+              ok = wait_load(seq, 6) && mbar_wait(sb + S::kPFull + 8 * b, (g / kSBufs) & 1, wc, 5);
+            else
+              ok = mbar_wait(sb + S::kPFull + 8 * b, (g / kSBufs) & 1, wc, 5) && wait_load(seq, 6);
+            ok = ok && (c.j != 0 || c.k == 0 || mbar_wait(sb + S::kOFree, static_cast<uint32_t>(c.k - 1) & 1, wc, 15));
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t st = seq % kStages;
+            const uint64_t dv = dv0 + st * kBlockStep;
+            const uint32_t tP = tmem + 128 * b;
+  #pragma unroll
+            for (int k16 = 0; k16 < 8; ++k16)
+              umma_ts(tO, tP + (k16 >> 2) * 64 + (k16 & 3) * 8, dv + static_cast<uint64_t>(k16 * (2048 >> 4)), idesc_pv,
+                      (c.j > 0 || k16 > 0) ? 1u : 0u);
+            umma_commit(sb + S::kKvEmpty + 8 * st);
+            umma_commit(sb + S::kPvDone + 8 * b);
+            if (c.j + 1 == c.it.kv_len) umma_commit(sb + S::kOFull);
+          }
+        }
+        // Drain: all MMAs issued by this thread complete before TMEM is freed.
+        const uint32_t drain = sb + (warp == kSWarp ? S::kDrainS : S::kDrain);
+        umma_commit(drain);
+        mbar_wait_drain(drain, 0, p.limit_ns);
+      }
+      __syncwarp();
     }
-    __syncwarp();
-  } else if (warp < 8) {
+  };
+  auto softmax_role = [&]() {
     setmaxnreg_inc<kRegsSoftmax>();
     // ------------------------------------------------------------ softmax + epilogue
     // Warps w and w+4 share the rows of TMEM lane quadrant w and take the blocks of
@@ -736,6 +744,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       cur.next(p);
     }
+  };
+  // Same work either way; the placement changes only how the compiler lays out and
+  // schedules the softmax loop.  Timed on B200 (launches alternating in one process,
+  // identical outputs): the tiled instantiation runs fastest with the softmax branch
+  // last; the mixed-layout one 2-3 % faster with it first, and the one-launch raster
+  // one faster with it first than last.
+  if constexpr (LAYOUT == kTiled) {
+    if (warp >= 8) other_roles(); else softmax_role();
+  } else {
+    if (warp < 8) softmax_role(); else other_roles();
   }
 
   tc_fence_before();
