@@ -2,8 +2,9 @@
 on CPU over randomised interleavings.
 
 Agents, as in the kernel: the producer (Q into two buffers; K and V into a ring
-in the order K0, K1, K2, V0, K3, V1, ...), the S issuer (S_g into TMEM buffer
-g mod 3 once P_g-3 V_g-3 has completed), the P V issuer, and two softmax warps
+in the order K0, K1, K2, V0, K3, V1, ... with B = 3 score buffers, K0 .. K3, V0,
+K4, V1, ... with B = 4), the S issuer (S_g into TMEM buffer g mod B once
+P_g-B V_g-B has completed), the P V issuer, and two softmax warps
 per lane quadrant that take alternate blocks, publish each block's outcome for
 the partner, may redo a block and rescale O, and share the epilogue through the
 row-sum exchange.  MMAs of one issuer execute in its issue order; the two
@@ -57,11 +58,14 @@ class Bar:
 
 class Forward:
     def __init__(self, items, seed, quads=2, stages=4, o_free=False, p_before_v=False, mutation=None,
-                 p_redo=0.25, early_waits=False):
+                 p_redo=0.25, early_waits=False, sbufs=3, p_tma=None):
         self.rng = random.Random(seed)
-        self.items, self.quads, self.stages = items, quads, stages
+        self.items, self.quads, self.stages, self.B = items, quads, stages, sbufs
         self.o_free, self.p_before_v, self.mutation, self.p_redo = o_free, p_before_v, mutation, p_redo
         self.early_waits = early_waits
+        # p_tma: when set, a step completes a pending TMA load with this probability (else
+        # another unit moves), so that loads can stay in flight for long stretches
+        self.p_tma = p_tma
         self.blocks = [(k, j) for k, n in enumerate(items) for j in range(n)]
         self.G = len(self.blocks)
         self.bars = {"OFull": Bar(1), "OFree": Bar(2 * quads)}
@@ -69,13 +73,13 @@ class Forward:
             self.bars[f"QFull{i}"], self.bars[f"QEmpty{i}"] = Bar(1), Bar(1)
         for s in range(stages):
             self.bars[f"KvFull{s}"], self.bars[f"KvEmpty{s}"] = Bar(1), Bar(1)
-        for b in range(3):
+        for b in range(sbufs):
             self.bars[f"SFull{b}"], self.bars[f"PFull{b}"], self.bars[f"PvDone{b}"] = Bar(1), Bar(quads), Bar(1)
         for q in range(quads):
             self.bars[f"Out{q}"], self.bars[f"Lx{q}"] = Bar(1), Bar(2)
         self.qbuf = [None, None]
         self.stage = [None] * stages                 # ("K", g) or ("V", g)
-        self.sbuf = [None] * 3                       # (block, quadrants whose rows already hold P)
+        self.sbuf = [None] * sbufs                   # (block, quadrants whose rows already hold P)
         self.O = None                                # (item, last block accumulated)
         self.outslot = {q: [None, None] for q in range(quads)}
         self.outcome_read = set()                    # (block, quadrant) outcome read by the partner
@@ -90,10 +94,10 @@ class Forward:
         self.tma = []
 
     def seq_k(self, g):
-        return g + max(0, g - 2)
+        return g + max(0, g - (self.B - 1))
 
     def seq_v(self, g):
-        return min(self.G + g, 2 * g + 3)
+        return min(self.G + g, 2 * g + self.B)
 
     # ------------------------------------------------------------ asynchronous units
     def issue(self, who, g):
@@ -106,7 +110,7 @@ class Forward:
     def execute(self, who):
         g = self.queues[who].pop(0)
         k, j = self.blocks[g]
-        b = g % 3
+        b = g % self.B
         if who == "S":
             assert self.qbuf[k % 2] == k, f"S_{g} reads the Q of item {self.qbuf[k % 2]}"
             assert self.stage[self.seq_k(g) % self.stages] == ("K", g), f"S_{g} reads a stage without K_{g}"
@@ -142,11 +146,11 @@ class Forward:
         return lambda: b.done(parity)
 
     def producer(self):
-        order = [("K", g) for g in range(min(3, self.G))]
+        order = [("K", g) for g in range(min(self.B, self.G))]
         for g in range(self.G):
             order.append(("V", g))
-            if g + 3 < self.G:
-                order.append(("K", g + 3))
+            if g + self.B < self.G:
+                order.append(("K", g + self.B))
         for n, (what, g) in enumerate(order):
             k, j = self.blocks[g]
             if what == "K" and j == 0:
@@ -163,14 +167,14 @@ class Forward:
 
     def s_issuer(self):
         for g, (k, j) in enumerate(self.blocks):
-            b, seq = g % 3, self.seq_k(g)
+            b, seq = g % self.B, self.seq_k(g)
             k_wait = self.wait(f"KvFull{seq % self.stages}", (seq // self.stages) & 1)
             if self.early_waits:       # K (and Q) before the buffer: they are off the chain
                 yield k_wait
                 if j == 0:
                     yield self.wait(f"QFull{k % 2}", (k // 2) & 1)
-            if g >= 3 and self.mutation != "no_pvdone_wait":
-                yield self.wait(f"PvDone{b}", ((g // 3) & 1) ^ 1)
+            if g >= self.B and self.mutation != "no_pvdone_wait":
+                yield self.wait(f"PvDone{b}", ((g // self.B) & 1) ^ 1)
             if not self.early_waits:
                 if j == 0:
                     yield self.wait(f"QFull{k % 2}", (k // 2) & 1)
@@ -183,12 +187,17 @@ class Forward:
 
     def pv_issuer(self):
         for g, (k, j) in enumerate(self.blocks):
-            b, seq = g % 3, self.seq_v(g)
+            b, seq = g % self.B, self.seq_v(g)
             v_wait = self.wait(f"KvFull{seq % self.stages}", (seq // self.stages) & 1)
-            p_wait = self.wait(f"PFull{b}", (g // 3) & 1)
-            # V first is safe once the stage's previous load is V_g-2, which this thread
-            # waited for itself (the steady part of the ring order, g >= 2)
-            v_first = not self.p_before_v or (self.early_waits and g >= 2 and seq == 2 * g + 3)
+            p_wait = self.wait(f"PFull{b}", (g // self.B) & 1)
+            # V first is safe where the load before V_g on its stage is one this thread
+            # waited for itself (V_g-stages/2, an even number of stages) or one that P_g-1
+            # implies (an earlier K): from g = 2 with three score buffers (four or eight
+            # stages), from g = 3 with four (six stages)
+            v_from = 2 if self.B == 3 else self.stages // 2
+            if self.mutation == "v_first_early":
+                v_from = 2
+            v_first = not self.p_before_v or (self.early_waits and g >= v_from and seq == 2 * g + self.B)
             for w in ((v_wait, p_wait) if v_first else (p_wait, v_wait)):
                 yield w
             if self.o_free and j == 0 and k > 0:
@@ -210,11 +219,11 @@ class Forward:
             self.outcome_read.add((gg, q))
 
         for g, (k, j) in enumerate(self.blocks):
-            b = g % 3
+            b = g % self.B
             if j == 0:
                 have_m = False
             if (g & 1) == h:
-                yield self.wait(f"SFull{b}", (g // 3) & 1)
+                yield self.wait(f"SFull{b}", (g // self.B) & 1)
                 mine = lambda: self.sbuf[b][0] == g and q not in self.sbuf[b][1]   # noqa: E731
                 assert mine(), f"warp ({q},{h}) reads S_{g} from a buffer holding {self.sbuf[b]}"
                 if j > 0 and not have_m:
@@ -223,7 +232,7 @@ class Forward:
                 if g > 0 and consumed != g - 1 and self.mutation != "no_outcome_read":
                     yield from read_outcome(g - 1)
                 if j > 0 and self.rng.random() < self.p_redo:        # redo with the exact max: rescale O
-                    yield self.wait(f"PvDone{(g - 1) % 3}", ((g - 1) // 3) & 1)
+                    yield self.wait(f"PvDone{(g - 1) % self.B}", ((g - 1) // self.B) & 1)
                     assert self.O == (k, g - 1), f"the rescale in block {g} sees O {self.O}"
                     yield lambda: True
                     assert self.O == (k, g - 1), f"O changed under the rescale in block {g}"
@@ -257,12 +266,17 @@ class Forward:
         for _ in range(max_steps):
             choices = [("agent", i) for i in range(len(agents)) if not done[i] and (waits[i] is None or waits[i]())]
             choices += [("mma", who) for who in ("S", "PV") if self.queues[who]]
-            choices += [("tma", i) for i in range(len(self.tma))]
-            if not choices:
+            tmas = [("tma", i) for i in range(len(self.tma))]
+            if not choices and not tmas:
                 assert all(done), "deadlock"
                 assert not any(self.commits.values())
                 return
-            what, x = self.rng.choice(choices)
+            if self.p_tma is None:
+                what, x = self.rng.choice(choices + tmas)
+            elif tmas and (not choices or self.rng.random() < self.p_tma):
+                what, x = self.rng.choice(tmas)
+            else:
+                what, x = self.rng.choice(choices)
             if what == "agent":
                 try:
                     waits[x] = next(agents[x])
@@ -280,13 +294,13 @@ class Forward:
         raise AssertionError("step limit")
 
 
-def _failures(n, seed, **kw):
+def _failures(n, seed, stages=(4, 8), **kw):
     rng = random.Random(seed)
     out = []
     for t in range(n):
         items = [rng.randint(1, 5) for _ in range(rng.randint(1, 5))]
         try:
-            Forward(items, seed=t, quads=rng.choice([1, 2]), stages=rng.choice([4, 8]), **kw).run()
+            Forward(items, seed=t, quads=rng.choice([1, 2]), stages=rng.choice(stages), **kw).run()
         except AssertionError as e:
             out.append(str(e))
     return out
@@ -297,6 +311,19 @@ def test_kernel_order_has_no_deadlock_and_no_stale_read():
     # last held V_g-2, and the S issuer's K and Q waits before its buffer wait
     assert _failures(3000, 1, o_free=True, p_before_v=True, early_waits=True) == []
     assert _failures(1000, 6, o_free=True, p_before_v=True) == []
+    # loads that stay in flight for long stretches (the early-pass hazards need them)
+    assert _failures(1500, 11, p_tma=0.05, o_free=True, p_before_v=True, early_waits=True) == []
+
+
+def test_four_buffers_need_v_first_only_past_half_the_ring():
+    # A variant with four score buffers of 96 keys and a six-stage ring (measured, not
+    # adopted): there V_2's stage last held K_2, which P V_1 does not imply, so waiting
+    # for V_2 before P_2 lets the parity wait pass early while K_2 is in flight; from
+    # g = 3 (half the ring) V first is safe.
+    kw = dict(stages=(6,), o_free=True, p_before_v=True, early_waits=True, sbufs=4, p_tma=0.05)
+    assert _failures(1500, 7, **kw) == []
+    fails = _failures(1500, 8, mutation="v_first_early", **kw)
+    assert fails and all(f.startswith(V_STAGE) for f in fails), fails[:3]
 
 
 def test_without_the_two_orderings_the_model_finds_both_hazards():
