@@ -467,7 +467,8 @@ def run_ours(args, cfg):
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(e2e_steps):
-        # the public host entry: heads in chunks, copies overlapped with the computation
+        # the public host entry (the C-ABI call sta_forward_host where the tile splits into
+        # 128-row slabs): heads in chunks, copies overlapped with the computation
         sta.sta_forward_from_host(q_h, k_h, v_h, out_h, grid, tile, wins, scale, heads_per_chunk=4)
     e1.record(stream)
     torch.cuda.synchronize()

@@ -258,6 +258,31 @@ sta_status sta_attention_fwd_mixed(const void* q, const void* k_tiled, const voi
                                    const sta_dim3* window_per_head, float scale, void* stream);
 
 /*
+ * STA forward from host memory to host memory.  The paper has no counterpart: it
+ * is the whole-job call for data that lives on the host.
+ *   q, k, v, out: host bf16 [batch, heads, T*H*W, d], raster order.  Pinned memory
+ *   (cudaHostAlloc, cudaHostRegister) lets the copies overlap the computation;
+ *   pageable memory works, with copies that do not.  out must not overlap q, k, v.
+ * The heads go through the current device in chunks of heads_per_chunk heads of one
+ * batch entry: while one chunk is computed (sta_tile_reorder_padded of k and v,
+ * then sta_attention_fwd_mixed), the next is copied in and the one before copied
+ * out, on three CUDA streams the library owns.  The work starts after what is
+ * already queued on `stream`, and the call returns once out holds the result.
+ * Per head the result equals sta_attention_fwd_mixed's on device tensors bit for
+ * bit (heads are independent).  The tile must split into 128-row slabs of whole
+ * frames, as for sta_attention_fwd_mixed; the grid may be padded.  The library
+ * keeps two sets of chunk buffers on the device (grown as needed, freed by
+ * sta_shutdown), and the call holds the library's lock throughout, so concurrent
+ * calls of the library from other threads wait for it.  A bounded wait that ran
+ * out is reported by sta_check_device_status.
+ * Errors: NULL, SHAPE, WINDOW, HEADDIM, ARG (batch, heads, scale or heads_per_chunk
+ * out of range), ALIAS, ARCH, CUDA.
+ */
+sta_status sta_forward_host(const void* q, const void* k, const void* v, void* out, int32_t batch, int32_t heads,
+                            int32_t d, sta_dim3 grid, sta_dim3 tile, const sta_dim3* window_per_head, float scale,
+                            int32_t heads_per_chunk, void* stream);
+
+/*
  * sta_attention_fwd without any device allocation by the library.  The paper has
  * no counterpart: this entry point exists for callers that cannot let a library
  * call cudaMalloc - code running inside a memory pool or arena it must not

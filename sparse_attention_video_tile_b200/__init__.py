@@ -65,6 +65,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "sta_attention_fwd_raster": (ctypes.c_int, [P, P, P, P, I32, I32, I32, D3, D3, ctypes.POINTER(D3), F, P]),
         "sta_attention_fwd_mixed": (ctypes.c_int, [P, P, P, P, I32, I32, I32, D3, D3, ctypes.POINTER(D3), F, P]),
         "sta_tile_reorder_padded": (ctypes.c_int, [P, P, I64, I32, D3, D3, P]),
+        "sta_forward_host": (ctypes.c_int, [P, P, P, P, I32, I32, I32, D3, D3, ctypes.POINTER(D3), F, I32, P]),
         "sta_attention_fwd_lse": (ctypes.c_int, [P, P, P, P, P, I32, I32, I32, D3, D3, ctypes.POINTER(D3), F, P]),
         "sta_attention_bwd": (ctypes.c_int, [P, P, P, P, P, P, P, P, P, I32, I32, I32, D3, D3, ctypes.POINTER(D3), F, P]),
         "sta_check_device_status": (ctypes.c_int, [P]),
@@ -460,13 +461,41 @@ def sta_forward_tokens(q, k, v, grid, tile, window_per_head, scale: Optional[flo
         return out
 
 
+def sta_forward_host(q_h, k_h, v_h, out_h, grid, tile, window_per_head, scale: Optional[float] = None,
+                     heads_per_chunk: int = 4, stream=None) -> None:
+    """The C-ABI call sta_forward_host on host tensors [B, heads, L, d] (bf16, raster
+    order, contiguous; pinned for overlapped copies): the library streams the heads
+    through the current device in chunks and returns once ``out_h`` holds the result."""
+    import torch
+    if q_h.dim() != 4:
+        raise ValueError("q must be [batch, heads, L, d]")
+    for name, t in (("k", k_h), ("v", v_h), ("out", out_h)):
+        if tuple(t.shape) != tuple(q_h.shape):
+            raise ValueError(f"{name} shape {tuple(t.shape)} differs from q {tuple(q_h.shape)}")
+    for name, t in (("q", q_h), ("k", k_h), ("v", v_h), ("out", out_h)):
+        if t.is_cuda or not t.is_contiguous() or t.dtype != torch.bfloat16:
+            raise ValueError(f"{name} must be a contiguous host bf16 tensor")
+    B, Hn, L, d = (int(x) for x in q_h.shape)
+    if len(window_per_head) != Hn:
+        raise ValueError("one window per head is required")
+    if L != int(np.prod([int(x) for x in grid])):
+        raise ValueError("L must equal T*H*W")
+    sc = 1.0 / float(d) ** 0.5 if scale is None else float(scale)
+    st = load_library().sta_forward_host(q_h.data_ptr(), k_h.data_ptr(), v_h.data_ptr(), out_h.data_ptr(), B, Hn, d,
+                                         _d3(grid), _d3(tile), _windows(window_per_head), sc, int(heads_per_chunk),
+                                         _stream(stream))
+    _check(st, "sta_forward_host")
+
+
 def sta_forward_from_host(q_h, k_h, v_h, out_h, grid, tile, window_per_head, scale: Optional[float] = None,
                           heads_per_chunk: int = 4, device=None) -> None:
     """STA forward from pinned host tensors [B, heads, L, d] (bf16, raster order)
     into the pinned host tensor ``out_h``, with the copies overlapped with the
-    computation: heads go through in chunks, and while one chunk is computed
-    (``sta_forward``) the next is copied in and the previous one copied out, on
-    three CUDA streams.  Per head the result equals ``sta_forward`` on device
+    computation: heads go through in chunks, and while one chunk is computed the
+    next is copied in and the previous one copied out, on three CUDA streams.  Where
+    the tile splits into 128-row slabs of whole frames (``raster_tile_ok``) this is
+    the C-ABI call ``sta_forward_host``; other tiles take the same pipeline built
+    here from ``sta_forward``.  Per head the result equals ``sta_forward`` on device
     tensors: heads are independent.  The work starts after what is already queued
     on the device's current stream (for example a copy that fills the inputs).
     Returns once ``out_h`` holds the output."""
@@ -486,7 +515,12 @@ def sta_forward_from_host(q_h, k_h, v_h, out_h, grid, tile, window_per_head, sca
         raise ValueError("heads_per_chunk must be positive")
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
     with torch.cuda.device(dev):
-        _forward_from_host_chunks(q_h, k_h, v_h, out_h, grid, tile, window_per_head, scale, heads_per_chunk, dev)
+        if raster_tile_ok(tile):
+            sta_forward_host(q_h, k_h, v_h, out_h, grid, tile, window_per_head, scale, heads_per_chunk,
+                             torch.cuda.current_stream(dev))
+        else:
+            _forward_from_host_chunks(q_h, k_h, v_h, out_h, grid, tile, window_per_head, scale, heads_per_chunk,
+                                      dev)
 
 
 def _forward_from_host_chunks(q_h, k_h, v_h, out_h, grid, tile, window_per_head, scale, heads_per_chunk, dev):

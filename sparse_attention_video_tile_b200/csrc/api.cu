@@ -58,7 +58,18 @@ struct CachedSchedule {
 using ScheduleKey = std::tuple<int32_t, int32_t, int32_t, int32_t, int32_t, int32_t, int32_t, int32_t, int32_t,
                                std::vector<int32_t>>;
 
+// Streams, events and chunk buffers of sta_forward_host (two slots of chunk buffers:
+// q, k, v and out in raster order, k and v in the padded tiled order).
+struct HostPipe {
+  cudaStream_t s_in = nullptr, s_run = nullptr, s_out = nullptr;
+  cudaEvent_t start = nullptr, copied[2] = {nullptr, nullptr}, computed[2] = {nullptr, nullptr},
+              drained[2] = {nullptr, nullptr};
+  uint8_t* buf = nullptr;
+  size_t bytes = 0;
+};
+
 struct DeviceState {
+  HostPipe pipe;
   int32_t* d_err = nullptr;  // bounded-wait status word
   float* d_dvec = nullptr;   // backward scratch: one float per query row
   size_t dvec_rows = 0;
@@ -536,6 +547,122 @@ sta_status sta_attention_fwd_mixed(const void* q, const void* k_tiled, const voi
   return e == cudaSuccess ? STA_OK : cuda_fail(e);
 }
 
+namespace {
+cudaError_t pipe_init(HostPipe* pp) {
+  if (pp->s_in) return cudaSuccess;
+  cudaError_t e = cudaSuccess;
+  for (cudaStream_t* s : {&pp->s_in, &pp->s_run, &pp->s_out})
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(s, cudaStreamNonBlocking);
+  for (cudaEvent_t* ev : {&pp->start, &pp->copied[0], &pp->copied[1], &pp->computed[0], &pp->computed[1],
+                          &pp->drained[0], &pp->drained[1]})
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
+  return e;
+}
+
+void pipe_free(HostPipe* pp) {
+  for (cudaStream_t s : {pp->s_in, pp->s_run, pp->s_out})
+    if (s) cudaStreamDestroy(s);
+  for (cudaEvent_t ev : {pp->start, pp->copied[0], pp->copied[1], pp->computed[0], pp->computed[1], pp->drained[0],
+                         pp->drained[1]})
+    if (ev) cudaEventDestroy(ev);
+  if (pp->buf) cudaFree(pp->buf);
+  *pp = HostPipe{};
+}
+}  // namespace
+
+sta_status sta_forward_host(const void* q, const void* k, const void* v, void* out, int32_t batch, int32_t heads,
+                            int32_t d, sta_dim3 grid, sta_dim3 tile, const sta_dim3* window_per_head, float scale,
+                            int32_t heads_per_chunk, void* stream) {
+  if (!q || !k || !v || !out || !window_per_head) return STA_ERR_NULL;
+  if (d != 64 && d != 128) return STA_ERR_HEADDIM;
+  Geometry g;
+  sta_status s = make_geometry_padded(grid, tile, &g);
+  if (s != STA_OK) return s;
+  if (!raster_tile_ok(g.tt, g.th, g.tw) || g.ntile % kBlockRows != 0) return STA_ERR_SHAPE;
+  if (batch < 1 || heads < 1 || static_cast<int64_t>(batch) * heads > (int64_t(1) << 24)) return STA_ERR_ARG;
+  if (heads_per_chunk < 1) return STA_ERR_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return STA_ERR_ARG;
+  for (int32_t h = 0; h < heads; ++h)
+    if (window_per_head[h].t < 1 || window_per_head[h].h < 1 || window_per_head[h].w < 1) return STA_ERR_WINDOW;
+  const int64_t head_bytes = g.L * d * 2;   // one (batch, head) slice, raster order
+  const int64_t bytes = static_cast<int64_t>(batch) * heads * head_bytes;
+  if (overlaps(out, q, bytes) || overlaps(out, k, bytes) || overlaps(out, v, bytes)) return STA_ERR_ALIAS;
+  int dev = 0;
+  if ((s = check_device(&dev)) != STA_OK) return s;
+
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState* st = nullptr;
+  if ((s = device_state(dev, &st)) != STA_OK) return s;
+  HostPipe& pp = st->pipe;
+  cudaError_t e = pipe_init(&pp);
+  if (e != cudaSuccess) return cuda_fail(e);
+  const int32_t hc = std::min(heads_per_chunk, heads);
+  const int64_t raster = hc * head_bytes, tiled = hc * g.Lpad * d * 2;
+  const size_t slot_bytes = static_cast<size_t>(4 * raster + 2 * tiled);   // q, k, v, out; k, v tiled
+  if (pp.bytes < 2 * slot_bytes) {
+    if ((e = cudaDeviceSynchronize()) != cudaSuccess) return cuda_fail(e);
+    if (pp.buf) cudaFree(pp.buf);
+    pp.buf = nullptr;
+    pp.bytes = 0;
+    if ((e = cudaMalloc(&pp.buf, 2 * slot_bytes)) != cudaSuccess) return cuda_fail(e);
+    pp.bytes = 2 * slot_bytes;
+  }
+  const uint8_t* hq = static_cast<const uint8_t*>(q);
+  const uint8_t* hk = static_cast<const uint8_t*>(k);
+  const uint8_t* hv = static_cast<const uint8_t*>(v);
+  uint8_t* hout = static_cast<uint8_t*>(out);
+  // the work starts after what is queued on the caller's stream
+  if ((e = cudaEventRecord(pp.start, static_cast<cudaStream_t>(stream))) != cudaSuccess) return cuda_fail(e);
+  for (cudaStream_t sx : {pp.s_in, pp.s_run, pp.s_out})
+    if ((e = cudaStreamWaitEvent(sx, pp.start, 0)) != cudaSuccess) return cuda_fail(e);
+  bool used[2] = {false, false};
+  int64_t i = 0;
+  for (int32_t b = 0; b < batch && e == cudaSuccess; ++b) {
+    for (int32_t h0 = 0; h0 < heads && e == cudaSuccess; h0 += hc, ++i) {
+      const int slot = static_cast<int>(i & 1);
+      const int32_t n = std::min(hc, heads - h0);
+      const int64_t off = (static_cast<int64_t>(b) * heads + h0) * head_bytes, len = n * head_bytes;
+      uint8_t* dq = pp.buf + slot * slot_bytes;
+      uint8_t *dk = dq + raster, *dv = dk + raster, *dout = dv + raster, *dkt = dout + raster, *dvt = dkt + tiled;
+      CachedSchedule* cs = nullptr;
+      if ((s = get_schedule(st, g, 1, n, window_per_head + h0, 1, &cs)) != STA_OK) break;
+      DeviceSchedule ds{cs->d_items, cs->d_kv_rows, cs->d_head_win, static_cast<int32_t>(cs->host.items.size()),
+                        false, cs->d_kv_mask_id, cs->d_kv_masks, static_cast<int32_t>(cs->host.kv_rows.size()),
+                        static_cast<int32_t>(cs->host.kv_masks.size() / 4)};
+      // copy in: the slot's inputs are free once its previous chunk was computed
+      if (used[slot] && (e = cudaStreamWaitEvent(pp.s_in, pp.computed[slot], 0)) != cudaSuccess) break;
+      if ((e = cudaMemcpyAsync(dq, hq + off, len, cudaMemcpyHostToDevice, pp.s_in)) != cudaSuccess ||
+          (e = cudaMemcpyAsync(dk, hk + off, len, cudaMemcpyHostToDevice, pp.s_in)) != cudaSuccess ||
+          (e = cudaMemcpyAsync(dv, hv + off, len, cudaMemcpyHostToDevice, pp.s_in)) != cudaSuccess ||
+          (e = cudaEventRecord(pp.copied[slot], pp.s_in)) != cudaSuccess)
+        break;
+      // compute: after the copy in, and once the slot's previous output was copied out
+      if ((e = cudaStreamWaitEvent(pp.s_run, pp.copied[slot], 0)) != cudaSuccess) break;
+      if (used[slot] && (e = cudaStreamWaitEvent(pp.s_run, pp.drained[slot], 0)) != cudaSuccess) break;
+      if ((e = launch_reorder_padded(dk, dkt, n, d, g, pp.s_run)) != cudaSuccess ||
+          (e = launch_reorder_padded(dv, dvt, n, d, g, pp.s_run)) != cudaSuccess ||
+          (e = launch_attention_mixed(dq, dkt, dvt, dout, 1, n, d, g, ds, scale, st->d_err, kWaitLimitNs,
+                                      pp.s_run)) != cudaSuccess ||
+          (e = cudaEventRecord(pp.computed[slot], pp.s_run)) != cudaSuccess)
+        break;
+      // copy out
+      if ((e = cudaStreamWaitEvent(pp.s_out, pp.computed[slot], 0)) != cudaSuccess ||
+          (e = cudaMemcpyAsync(hout + off, dout, len, cudaMemcpyDeviceToHost, pp.s_out)) != cudaSuccess ||
+          (e = cudaEventRecord(pp.drained[slot], pp.s_out)) != cudaSuccess)
+        break;
+      used[slot] = true;
+    }
+  }
+  // every queued copy and kernel completes before the call returns, also after an error
+  const cudaError_t e_in = cudaStreamSynchronize(pp.s_in), e_run = cudaStreamSynchronize(pp.s_run),
+                    e_out = cudaStreamSynchronize(pp.s_out);
+  if (s != STA_OK) return s;
+  if (e != cudaSuccess) return cuda_fail(e);
+  for (cudaError_t ex : {e_in, e_run, e_out})
+    if (ex != cudaSuccess) return cuda_fail(ex);
+  return STA_OK;
+}
+
 sta_status sta_check_device_status(void* stream) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -595,6 +722,7 @@ void sta_shutdown(void) {
     if (kv.second.d_dvec) cudaFree(kv.second.d_dvec);
     kv.second.d_dvec = nullptr;
     kv.second.dvec_rows = 0;
+    pipe_free(&kv.second.pipe);
   }
   g_devices.clear();
   noalloc_reset();

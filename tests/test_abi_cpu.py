@@ -179,6 +179,7 @@ def test_no_cpu_fallback_without_gpu(lib):
     assert _call_tokens(lib, 0x100000, 0x100000 + 64 * 1024, heads=1) in (7, 8)
     assert _call_attn(lib) in (7, 8)
     assert _call_bwd(lib) in (7, 8)
+    assert _call_host(lib) in (7, 8)
 
 
 def test_python_paths_refuse_cpu_tensors(lib):
@@ -269,3 +270,21 @@ def test_padded_reorder_and_mixed_validation_codes(lib):
         # valid arguments and no GPU: a CUDA/architecture error, never a host computation
         assert pad(A, B) in (7, 8)
         assert _call_mixed(lib) in (7, 8)
+
+
+def _call_host(lib, q=0x1000000, k=0x2000000, v=0x3000000, out=0x4000000, batch=1, heads=1, d=128,
+               grid=(12, 24, 40), tile=(6, 8, 8), windows=((1, 3, 3),), scale=0.1, chunk=4):
+    return lib.sta_forward_host(q, k, v, out, batch, heads, d, sta._d3(grid), sta._d3(tile), sta._windows(windows),
+                                ctypes.c_float(scale), chunk, None)
+
+
+def test_forward_host_validation_codes(lib):
+    codes = {name: code for code, name in sta.STATUS_NAMES.items()}
+    assert _call_host(lib, q=0) == codes["STA_ERR_NULL"]
+    assert _call_host(lib, d=96) == codes["STA_ERR_HEADDIM"]
+    assert _call_host(lib, grid=(4, 8, 8), tile=(2, 4, 4)) == codes["STA_ERR_SHAPE"]   # no 128-row slabs
+    assert _call_host(lib, windows=((0, 3, 3),)) == codes["STA_ERR_WINDOW"]
+    assert _call_host(lib, chunk=0) == codes["STA_ERR_ARG"]
+    assert _call_host(lib, batch=0) == codes["STA_ERR_ARG"]
+    assert _call_host(lib, scale=-1.0) == codes["STA_ERR_ARG"]
+    assert _call_host(lib, out=0x1000000 + 64) == codes["STA_ERR_ALIAS"]

@@ -456,3 +456,16 @@ def test_forward_from_host_equals_device_forward():
     sta.sta_forward_from_host(qh, kh, vh, out_h, cfg.grid, cfg.tile, cfg.windows, cfg.scale, heads_per_chunk=2)
     assert sta.sta_check_device_status() == sta.STA_OK
     assert torch.equal(out_h, want.cpu())
+
+
+def test_forward_host_pageable_padded_latent():
+    """The C-ABI host entry on pageable host memory (copies that do not overlap) and a
+    latent that is not a tile multiple (padded inside, real tokens only in and out),
+    three heads in chunks of two: the device forward's bits, head by head."""
+    cfg = W.custom_config("host_padded", 1, 3, 128, (11, 22, 37), (6, 8, 8), [(1, 3, 3), (3, 3, 3), (1, 1, 1)])
+    q, k, v = W.make_qkv(cfg, 21)
+    want = sta.sta_forward(q.cuda(), k.cuda(), v.cuda(), cfg.grid, cfg.tile, cfg.windows, cfg.scale)
+    out_h = torch.empty(q.shape, dtype=q.dtype)
+    sta.sta_forward_host(q, k, v, out_h, cfg.grid, cfg.tile, cfg.windows, cfg.scale, heads_per_chunk=2)
+    assert sta.sta_check_device_status() == sta.STA_OK
+    assert torch.equal(out_h, want.cpu())
