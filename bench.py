@@ -461,6 +461,8 @@ def run_ours(args, cfg):
 
     # ---- end to end through the public API with host buffers
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
+    # one untimed call: the library sets up its chunk buffers and streams on the first
+    sta.sta_forward_from_host(q_h, k_h, v_h, out_h, grid, tile, wins, scale, heads_per_chunk=4)
     barrier()
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
