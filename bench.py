@@ -42,8 +42,8 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # workload, from an ncu capture of the 4-head case of that workload (scaled by 6 to 24 heads:
 # traffic is per head).  Valid only for the kernel source it was taken on, identified by the
 # SHA-1 of attention.cu and ptx.cuh (an edit of comments alone carries the figures over).
-PROFILED_TRAFFIC = {"sha1": "a25276ed329e597c71f1f0015f70c3c586bdf0e6", "workload": "hunyuan",
-                    "bytes_per_launch": {"mixed": 6 * (361.169664e6 + 103.045120e6),
+PROFILED_TRAFFIC = {"sha1": "a40d341bba712b1f4cd6c88627097a079a90f28c", "workload": "hunyuan",
+                    "bytes_per_launch": {"mixed": 6 * (359.788800e6 + 103.340800e6),
                                          "three_call": 6 * (357.326336e6 + 103.657216e6)}}
 
 

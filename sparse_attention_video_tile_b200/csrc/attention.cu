@@ -38,7 +38,7 @@
 //     bf16 rows, each warp half of the head dimension;
 //   * warpgroup 2 (warps 8-11: the producer, the two issuers and one idle warp)
 //     lowers its register count with setmaxnreg and the two softmax warpgroups
-//     raise theirs to 224 (216 in the mixed-layout kernel), so that a softmax
+//     raise theirs to 224 (200 in the mixed-layout kernel), so that a softmax
 //     thread holds half a row of S, the row's P and its state without spilling.
 //
 // Every barrier that is waited on with a parity can never run two phases ahead
@@ -82,7 +82,7 @@ constexpr bool kChecks = STA_DEVICE_CHECKS != 0;
 
 constexpr int kThreads = 384;       // warps 0-7 softmax + epilogue, 8 producer, 9-10 MMA issuers, 11 idle
 constexpr int kRegsSoftmax = 224;   // setmaxnreg: warpgroups 0-1 (softmax) raise, warpgroup 2 lowers
-constexpr int kRegsOther = 56;      // (per layout in the kernel: 216 and 64 for the mixed layout)
+constexpr int kRegsOther = 56;      // (per layout in the kernel: 200 and 96 for the mixed layout)
 constexpr int kRegsAtLaunch = 168;  // 65536 / 384 rounded down to a multiple of 8
 constexpr int kProducerWarp = 8;
 constexpr int kPvWarp = 9;          // issues O += P V; also owns the TMEM allocation
@@ -251,10 +251,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr uint32_t kBlockBytes = S::kBlockBytes;
 
   // Register split per layout, timed on B200 like the branch placement below: the
-  // mixed-layout instantiation runs about 2 % faster with 216 / 64 than with 224 / 56.
-  // The split must fit the registers the block was launched with.
-  constexpr int kRegsSm = LAYOUT == kMixed ? 216 : kRegsSoftmax;
-  constexpr int kRegsOt = LAYOUT == kMixed ? 64 : kRegsOther;
+  // mixed-layout instantiation runs about 3 % faster with 200 / 96 than with 224 / 56
+  // (216 / 64: 2 %; 208 / 80 and 232 / 40 slower).  The split must fit the registers
+  // the block was launched with.
+  constexpr int kRegsSm = LAYOUT == kMixed ? 200 : kRegsSoftmax;
+  constexpr int kRegsOt = LAYOUT == kMixed ? 96 : kRegsOther;
   static_assert(256 * kRegsSm + 128 * kRegsOt <= kThreads * kRegsAtLaunch, "register split above the launch allocation");
   // The two role branches, softmax warps and the rest, as lambdas, so that the order in
   // which they are placed in the code can be chosen per layout (end of the kernel).
