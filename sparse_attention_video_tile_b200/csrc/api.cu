@@ -157,6 +157,11 @@ sta_status get_schedule(DeviceState* st, const Geometry& g, int32_t batch, int32
     return cuda_fail(e);
   }
   st->schedules.emplace_front(std::move(key), std::move(cs));
+  if (st->schedules.size() > kMaxCachedSchedules) {
+    // a kernel queued earlier on any stream may still read the evicted schedule's arrays
+    cudaError_t es = cudaDeviceSynchronize();
+    if (es != cudaSuccess) return cuda_fail(es);
+  }
   while (st->schedules.size() > kMaxCachedSchedules) {
     free_schedule(st->schedules.back().second.get());
     st->schedules.pop_back();

@@ -469,3 +469,25 @@ def test_forward_host_pageable_padded_latent():
     sta.sta_forward_host(q, k, v, out_h, cfg.grid, cfg.tile, cfg.windows, cfg.scale, heads_per_chunk=2)
     assert sta.sta_check_device_status() == sta.STA_OK
     assert torch.equal(out_h, want.cpu())
+
+
+def test_schedule_cache_eviction_with_launches_in_flight():
+    """More configurations than the library's schedule cache holds, launched back to back
+    with one synchronize at the end: evicting a schedule must not free arrays that a
+    queued kernel still reads.  Every output is checked against the oracle."""
+    grids = [(4, 8, 8), (6, 8, 8), (4, 12, 8)]
+    windows = [(a, b, c) for a in (1, 3) for b in (1, 3) for c in (1, 3)]
+    runs = []
+    for gi, grid in enumerate(grids):
+        for wi, win in enumerate(windows):
+            cfg = W.custom_config(f"evict_{gi}_{wi}", 1, 1, 64, grid, (2, 4, 4), [win])
+            q, k, v = W.make_qkv(cfg, 100 + 8 * gi + wi)
+            out = sta.sta_forward(q.cuda(), k.cuda(), v.cuda(), cfg.grid, cfg.tile, cfg.windows, cfg.scale)
+            runs.append((cfg, q, k, v, out))
+    assert len(runs) > 16
+    torch.cuda.synchronize()
+    assert sta.sta_check_device_status() == sta.STA_OK
+    for cfg, q, k, v, out in runs:
+        want = O.sta_attention_head(q[0, 0].double().numpy(), k[0, 0].double().numpy(),
+                                    v[0, 0].double().numpy(), cfg.grid, cfg.tile, cfg.windows[0], cfg.scale)
+        _compare(out[0, 0].float().cpu().numpy(), want, cfg.name)
