@@ -31,6 +31,9 @@
  * Ownership and execution: the caller owns every device buffer.  Calls are
  * asynchronous on the given stream (a cudaStream_t passed as void*, NULL = the
  * legacy default stream), out of place, and never synchronise unless stated.
+ * The attention calls build a work schedule per configuration on first use
+ * (a blocking upload) and keep the 16 most recently used; evicting an older one
+ * synchronises the device first, since a queued kernel may still read it.
  * On an invalid argument a call returns an error before touching any buffer or
  * the device.  Nothing is printed.
  */
