@@ -361,6 +361,22 @@ def pin_lse_matches_library(o):
         assert np.max(np.abs(got - want)) < 1e-12
 
 
+def pin_lse_closed_forms(o):
+    """q = 0 makes every allowed score zero, so lse_i = log(number of keys in the window)
+    = log(Ntile * prod min(w, n)); adding one vector c to every key shifts row i's scores,
+    and so its lse, by scale * q_i . c."""
+    for grid, tile, window in [((4, 8, 8), (2, 4, 4), (1, 3, 5)), ((6, 4, 10), (2, 2, 2), (3, 1, 2))]:
+        L, d, scale = int(np.prod(grid)), 5, 0.8
+        n = [g // t for g, t in zip(grid, tile)]
+        count = int(np.prod(tile)) * int(np.prod([min(w, m) for w, m in zip(window, n)]))
+        q, k, _ = _rand_qkv(L, d, seed=L + 1)
+        got = o.sta_lse_head(np.zeros_like(q), k, grid, tile, window, scale)
+        assert np.max(np.abs(got - np.log(count))) < 1e-12
+        c = np.linspace(-1.0, 1.5, d)
+        shifted = o.sta_lse_head(q, k + c, grid, tile, window, scale)
+        assert np.max(np.abs(shifted - o.sta_lse_head(q, k, grid, tile, window, scale) - scale * (q @ c))) < 1e-10
+
+
 def _autograd_reference(q, k, v, do, mask, scale):
     """dq, dk, dv of scaled_dot_product_attention with a boolean mask, by torch autograd."""
     t = [torch.from_numpy(np.ascontiguousarray(x)).clone().requires_grad_(True) for x in (q, k, v)]
@@ -437,6 +453,7 @@ ALL_PINS = [
     pin_padding_equals_explicit_padded_grid,
     pin_padding_is_noop_on_tile_multiples,
     pin_lse_matches_library,
+    pin_lse_closed_forms,
     pin_backward_equals_autograd,
     pin_backward_finite_differences,
     pin_backward_closed_forms,
